@@ -1,0 +1,442 @@
+/*
+ * fp8attn CPU oracle -- TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, obviously-correct restatement of what the FP8 attention
+ * path computes, used by the tests, by the smoke check and by the benchmark's
+ * CPU-baseline leg.  It shares no code, header, table or constant with the
+ * CUDA library and must never be linked into, or called by, the product path.
+ *
+ * Sources (web pages on on-the-fly FP8 attention quantisation):
+ *   [vLLM-ViT]  vLLM docs, "FP8 ViT encoder attention" -- usage section:
+ *               a 16-entry circular buffer of observed Q/K/V amax values
+ *               drives the per-forward scale; static per-layer {q,k,v}
+ *               scale file; saved scales multiplied by a save margin
+ *               (default 1.5); scale-file format section.
+ *   [vLLM-Omni] vLLM-Omni docs, "Quantized KV Cache" -- overview (Q/K/V
+ *               quantised dynamically before the FA operator) and the
+ *               parameters table (skip selectors).
+ *   [Ascend]    Ascend quantisation chapter -- names FP8 E4M3 / E5M2.
+ * The pages leave the E4M3 bit layout, rounding, the scale formula, the ring
+ * reduction and the P (softmax probability) rule open; the readings used here
+ * are the plainest ones and are written beside each function:
+ *   - E4M3 is the OCP 8-bit "FN" format (bias 7, no infinities, 0x7F/0xFF
+ *     NaN, max 448); encoding rounds to nearest, ties to even, and saturates
+ *     to +-448 (satfinite); NaN encodes as 0x7F.
+ *   - amax is max |x| over the valid (unpadded) tokens; NaN is ignored.
+ *   - the ring is reduced with max, the current pass is pushed first
+ *     ("current-inclusive"), and the bound A gives qs = fl32(448/A),
+ *     ds = fl32(A/448); A == 0 gives qs = ds = 1.
+ *   - static values are bounds A in activation units (the margin is applied
+ *     when they are saved, never again on load).
+ *   - attention quantises p = exp(s - M) (M = the row's final max) as
+ *     e4m3(256 p)/256 for the PV product and normalises by l = sum of the
+ *     unquantised p.
+ *
+ * Floating point: quantisation follows the kernel's stated fp32 rules (one
+ * fp32 RN multiply, one fp32 RN division), attention is evaluated in fp64.
+ * Build with -O2 -ffp-contract=off and no fast-math.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <pthread.h>
+#include <unistd.h>
+
+/* ------------------------------------------------------------------ */
+/* bf16                                                                */
+/* ------------------------------------------------------------------ */
+
+static float bf16_to_f32(uint16_t b) {
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* ------------------------------------------------------------------ */
+/* E4M3 ([Ascend] names the format; layout from the OCP FP8 spec)      */
+/* ------------------------------------------------------------------ */
+
+/* Value of an E4M3 (FN) code: sign, 4-bit exponent (bias 7), 3-bit mantissa.
+ * Exponent field 0 is subnormal (m/8 * 2^-6); field 15 with mantissa 7 is NaN.
+ * There is no infinity. */
+double or_e4m3_value(uint8_t code) {
+    int s = (code >> 7) & 1;
+    int e = (code >> 3) & 15;
+    int m = code & 7;
+    double mag;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        mag = ldexp((double)m, -9);          /* (m/8) * 2^-6 */
+    else
+        mag = ldexp(8.0 + (double)m, e - 10); /* (1 + m/8) * 2^(e-7) */
+    return s ? -mag : mag;
+}
+
+/* Encode a real number to E4M3: round to nearest, ties to the even
+ * mantissa, saturate magnitudes >= 448 to +-448, NaN -> 0x7F.  The sign is
+ * kept, so negative values that round to zero give 0x80. */
+uint8_t or_e4m3_encode(double y) {
+    uint8_t sign;
+    double a, step, r, n, frac;
+    int e2, efield, mant;
+    if (isnan(y)) return 0x7F;
+    sign = signbit(y) ? 0x80 : 0x00;
+    a = fabs(y);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+    if (a < ldexp(1.0, -6)) {
+        /* subnormal binade: spacing 2^-9 */
+        step = ldexp(1.0, -9);
+        efield = 0;
+    } else {
+        /* a in [2^E, 2^(E+1)) with E = e2 - 1; spacing 2^(E-3) */
+        (void)frexp(a, &e2);
+        step = ldexp(1.0, (e2 - 1) - 3);
+        efield = (e2 - 1) + 7;
+    }
+    r = a / step;              /* exact: division by a power of two */
+    n = floor(r);
+    frac = r - n;
+    if (frac > 0.5 || (frac == 0.5 && fmod(n, 2.0) == 1.0)) n += 1.0;
+    if (efield == 0) {
+        /* n in [0, 8]; n == 8 is the smallest normal 2^-6 */
+        if (n >= 8.0) { efield = 1; mant = 0; }
+        else mant = (int)n;
+    } else {
+        /* n in [8, 16]; n == 16 carries into the next binade */
+        if (n >= 16.0) { efield += 1; mant = 0; }
+        else mant = (int)n - 8;
+    }
+    /* a < 448 so rounding never reaches 480 (the NaN pattern) */
+    return (uint8_t)(sign | (efield << 3) | mant);
+}
+
+/* Bulk encode of fp32 inputs (used by the exhaustive cast tests). */
+void or_e4m3_encode_f32_array(const float* y, int64_t n, uint8_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = or_e4m3_encode((double)y[i]);
+}
+
+/* Bulk decode. */
+void or_e4m3_value_array(const uint8_t* c, int64_t n, double* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = or_e4m3_value(c[i]);
+}
+
+/* ------------------------------------------------------------------ */
+/* Valid-token addressing ("unpadding", [vLLM-ViT] notes: quant        */
+/* launches + unpadding).  Output row t of sequence b reads source row */
+/* t (packed) or src_seq_start[b] + (t - cu[b]) (padded source).       */
+/* ------------------------------------------------------------------ */
+
+static int64_t src_row_of(int64_t t, const int32_t* cu, int B,
+                          const int32_t* src_seq_start) {
+    int b;
+    if (!src_seq_start) return t;
+    for (b = 0; b < B; ++b)
+        if (t >= cu[b] && t < cu[b + 1]) break;
+    return (int64_t)src_seq_start[b] + (t - cu[b]);
+}
+
+/* Simple parallel-for over token ranges (pthreads). */
+typedef struct {
+    void (*fn)(void* ctx, int64_t t0, int64_t t1, int worker);
+    void* ctx;
+    int64_t T;
+    int nthreads;
+    int worker;
+} pf_arg;
+
+static void* pf_thread(void* p) {
+    pf_arg* a = (pf_arg*)p;
+    int64_t chunk = (a->T + a->nthreads - 1) / a->nthreads;
+    int64_t t0 = (int64_t)a->worker * chunk, t1 = t0 + chunk;
+    if (t1 > a->T) t1 = a->T;
+    if (t0 < t1) a->fn(a->ctx, t0, t1, a->worker);
+    return NULL;
+}
+
+static int parallel_for(int64_t T, int nthreads,
+                        void (*fn)(void*, int64_t, int64_t, int), void* ctx) {
+    pthread_t th[256];
+    pf_arg args[256];
+    int i;
+    if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    for (i = 0; i < nthreads; ++i) {
+        args[i].fn = fn; args[i].ctx = ctx; args[i].T = T;
+        args[i].nthreads = nthreads; args[i].worker = i;
+        pthread_create(&th[i], NULL, pf_thread, &args[i]);
+    }
+    for (i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    return nthreads;
+}
+
+typedef struct {
+    const uint16_t* x;
+    int64_t tok_stride, head_stride;
+    const int32_t* src_seq_start;
+    const int32_t* cu;
+    int B, H, D;
+    float qs;
+    uint8_t* out;
+    float part_amax[256];
+    int part_inf[256];
+} tensor_job;
+
+/* amax = max |x| over every valid token, head and channel of one tensor.
+ * NaN elements are ignored; an infinity is recorded as non-finite. */
+static void amax_range(void* p, int64_t t0, int64_t t1, int w) {
+    tensor_job* j = (tensor_job*)p;
+    float amax = 0.0f;
+    int inf = 0, h, d;
+    int64_t t;
+    for (t = t0; t < t1; ++t) {
+        int64_t row = src_row_of(t, j->cu, j->B, j->src_seq_start);
+        for (h = 0; h < j->H; ++h)
+            for (d = 0; d < j->D; ++d) {
+                float v = bf16_to_f32(j->x[row * j->tok_stride + h * j->head_stride + d]);
+                float a;
+                if (isnan(v)) continue;
+                a = fabsf(v);
+                if (isinf(a)) inf = 1;
+                if (a > amax) amax = a;
+            }
+    }
+    j->part_amax[w] = amax;
+    j->part_inf[w] = inf;
+}
+
+float or_amax_bf16(const uint16_t* x, int64_t tok_stride, int64_t head_stride,
+                   const int32_t* src_seq_start, const int32_t* cu, int B,
+                   int H, int D, int* nonfinite, int nthreads) {
+    tensor_job j;
+    float amax = 0.0f;
+    int n, i;
+    memset(&j, 0, sizeof(j));
+    j.x = x; j.tok_stride = tok_stride; j.head_stride = head_stride;
+    j.src_seq_start = src_seq_start; j.cu = cu; j.B = B; j.H = H; j.D = D;
+    n = parallel_for(cu[B], nthreads, amax_range, &j);
+    *nonfinite = 0;
+    for (i = 0; i < n; ++i) {
+        if (j.part_amax[i] > amax) amax = j.part_amax[i];
+        if (j.part_inf[i]) *nonfinite = 1;
+    }
+    return amax;
+}
+
+/* Cast: code = E4M3(fl32(x * qs)) -- one fp32 RN multiply, then RNE encode.
+ * Output is packed [T][H][D]. */
+static void quant_range(void* p, int64_t t0, int64_t t1, int w) {
+    tensor_job* j = (tensor_job*)p;
+    int64_t t;
+    int h, d;
+    (void)w;
+    for (t = t0; t < t1; ++t) {
+        int64_t row = src_row_of(t, j->cu, j->B, j->src_seq_start);
+        for (h = 0; h < j->H; ++h)
+            for (d = 0; d < j->D; ++d) {
+                float v = bf16_to_f32(j->x[row * j->tok_stride + h * j->head_stride + d]);
+                float y = v * j->qs;
+                j->out[(t * j->H + h) * (int64_t)j->D + d] = or_e4m3_encode((double)y);
+            }
+    }
+}
+
+void or_quantize_bf16(const uint16_t* x, int64_t tok_stride, int64_t head_stride,
+                      const int32_t* src_seq_start, const int32_t* cu, int B,
+                      int H, int D, float qs, uint8_t* out, int nthreads) {
+    tensor_job j;
+    memset(&j, 0, sizeof(j));
+    j.x = x; j.tok_stride = tok_stride; j.head_stride = head_stride;
+    j.src_seq_start = src_seq_start; j.cu = cu; j.B = B; j.H = H; j.D = D;
+    j.qs = qs; j.out = out;
+    parallel_for(cu[B], nthreads, quant_range, &j);
+}
+
+/* ------------------------------------------------------------------ */
+/* Amax ring and scales ([vLLM-ViT] usage: 16 observed amax values     */
+/* drive the per-forward scale; save margin 1.5).                      */
+/* ------------------------------------------------------------------ */
+
+#define OR_RING 16
+
+typedef struct {
+    float slot[OR_RING];
+    uint32_t head;   /* next slot to write */
+    uint32_t count;  /* filled slots, <= 16 */
+} or_ring;
+
+void or_ring_reset(or_ring* r) { memset(r, 0, sizeof(*r)); }
+
+/* Push one observed amax into the circular buffer. */
+void or_ring_push(or_ring* r, float amax) {
+    r->slot[r->head] = amax;
+    r->head = (r->head + 1) % OR_RING;
+    if (r->count < OR_RING) r->count += 1;
+}
+
+/* Bound A = max over the filled slots (0 for an empty ring). */
+float or_ring_bound(const or_ring* r) {
+    float a = 0.0f;
+    uint32_t i;
+    for (i = 0; i < r->count; ++i)
+        if (r->slot[i] > a) a = r->slot[i];
+    return a;
+}
+
+/* qs = fl32(448 / A), ds = fl32(A / 448); A == 0 -> 1, 1. */
+void or_scales_from_bound(float A, float* qs, float* ds) {
+    if (A == 0.0f) {
+        *qs = 1.0f;
+        *ds = 1.0f;
+        return;
+    }
+    *qs = 448.0f / A;
+    *ds = A / 448.0f;
+}
+
+/* One dynamic pass for one tensor: the current amax is pushed first (unless
+ * it is not finite, in which case the ring is left as it was), then the
+ * scales come from the ring's bound. */
+void or_dynamic_step(or_ring* r, float amax, int nonfinite, float* qs, float* ds) {
+    if (!nonfinite) or_ring_push(r, amax);
+    or_scales_from_bound(or_ring_bound(r), qs, ds);
+}
+
+/* Exported static value = fl32(bound * margin). */
+float or_export_value(const or_ring* r, float margin) {
+    return or_ring_bound(r) * margin;
+}
+
+/* ------------------------------------------------------------------ */
+/* Attention (fp64), non-causal, per sequence of cu_seqlens            */
+/* ([vLLM-Omni] overview: Q/K/V quantised before the FA operator;      */
+/* eligible forwards are full, non-causal attention).                  */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    int kind;                 /* 0 = fp8 codes, 1 = bf16 */
+    const void* q;
+    const void* k;
+    const void* v;
+    const int32_t* cu;
+    int B, H, D;
+    double ds_q, ds_k, ds_v;
+    double scale;             /* softmax scale (1/sqrt(D) by default) */
+    int pquant;               /* 0: p~ = p, 1: p~ = e4m3(256 p)/256 */
+    int lrule;                /* 0: l = sum p, 1: l = sum p~ */
+    const int64_t* rows;      /* token indices to evaluate (or NULL: all) */
+    int64_t nrows;
+    double* out;              /* [nrows][H][D] */
+    int64_t next;             /* work counter (rows*H items) */
+    pthread_mutex_t lock;
+} att_job;
+
+static double elem(const att_job* j, const void* base, int64_t t, int h, int d) {
+    int64_t idx = ((int64_t)t * j->H + h) * j->D + d;
+    if (j->kind == 0) return or_e4m3_value(((const uint8_t*)base)[idx]);
+    return (double)bf16_to_f32(((const uint16_t*)base)[idx]);
+}
+
+static void attend_one(const att_job* j, int64_t ri, int h, double* s_buf) {
+    int64_t t = j->rows ? j->rows[ri] : ri;
+    int b, d;
+    int64_t k0, k1, kk;
+    double M = -INFINITY, l = 0.0;
+    double* o = j->out + (ri * j->H + h) * (int64_t)j->D;
+    double dsq = j->kind == 0 ? j->ds_q : 1.0;
+    double dsk = j->kind == 0 ? j->ds_k : 1.0;
+    double dsv = j->kind == 0 ? j->ds_v : 1.0;
+    for (b = 0; b < j->B; ++b)
+        if (t >= j->cu[b] && t < j->cu[b + 1]) break;
+    k0 = j->cu[b];
+    k1 = j->cu[b + 1];
+    /* scores: dot of decoded values (exact in fp64 for E4M3), then scales */
+    for (kk = k0; kk < k1; ++kk) {
+        double acc = 0.0;
+        for (d = 0; d < j->D; ++d) acc += elem(j, j->q, t, h, d) * elem(j, j->k, kk, h, d);
+        s_buf[kk - k0] = acc * dsq * dsk * j->scale;
+        if (s_buf[kk - k0] > M) M = s_buf[kk - k0];
+    }
+    for (d = 0; d < j->D; ++d) o[d] = 0.0;
+    for (kk = k0; kk < k1; ++kk) {
+        double p = exp(s_buf[kk - k0] - M);
+        double pt = p;
+        if (j->pquant) pt = or_e4m3_value(or_e4m3_encode(256.0 * p)) / 256.0;
+        l += j->lrule ? pt : p;
+        for (d = 0; d < j->D; ++d) o[d] += pt * elem(j, j->v, kk, h, d);
+    }
+    for (d = 0; d < j->D; ++d) o[d] = o[d] * dsv / l;
+}
+
+static void* att_worker(void* arg) {
+    att_job* j = (att_job*)arg;
+    int64_t maxlen = 0, total = j->nrows * j->H;
+    int b;
+    double* s_buf;
+    for (b = 0; b < j->B; ++b)
+        if (j->cu[b + 1] - j->cu[b] > maxlen) maxlen = j->cu[b + 1] - j->cu[b];
+    s_buf = (double*)malloc(sizeof(double) * (size_t)(maxlen > 0 ? maxlen : 1));
+    for (;;) {
+        int64_t w;
+        pthread_mutex_lock(&j->lock);
+        w = j->next++;
+        pthread_mutex_unlock(&j->lock);
+        if (w >= total) break;
+        attend_one(j, w / j->H, (int)(w % j->H), s_buf);
+    }
+    free(s_buf);
+    return NULL;
+}
+
+static int run_attention(att_job* j, int nthreads) {
+    pthread_t th[256];
+    int i;
+    if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if (!j->rows) j->nrows = j->cu[j->B];
+    j->next = 0;
+    pthread_mutex_init(&j->lock, NULL);
+    for (i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, att_worker, j);
+    for (i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    pthread_mutex_destroy(&j->lock);
+    return nthreads;
+}
+
+/* FP8 attention on E4M3 codes [T][H][D] with per-tensor descales.
+ * o_i = (sum_j p~_ij dec(v_j)) * ds_v / l_i with p_ij = exp(s_ij - M_i),
+ * s_ij = (sum_d dec(q_id) dec(k_jd)) * ds_q * ds_k * scale.
+ * Returns the number of threads used. */
+int or_attention_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
+                     const int32_t* cu, int B, int H, int D,
+                     double ds_q, double ds_k, double ds_v, double scale,
+                     int pquant, int lrule, const int64_t* rows, int64_t nrows,
+                     double* out, int nthreads) {
+    att_job j;
+    memset(&j, 0, sizeof(j));
+    j.kind = 0;
+    j.q = q8; j.k = k8; j.v = v8;
+    j.cu = cu; j.B = B; j.H = H; j.D = D;
+    j.ds_q = ds_q; j.ds_k = ds_k; j.ds_v = ds_v; j.scale = scale;
+    j.pquant = pquant; j.lrule = lrule;
+    j.rows = rows; j.nrows = nrows; j.out = out;
+    return run_attention(&j, nthreads);
+}
+
+/* Native-dtype attention for skipped layers ([vLLM-Omni] parameters:
+ * listed layers keep the native dtype): bf16 inputs, no quantisation. */
+int or_attention_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                      const int32_t* cu, int B, int H, int D, double scale,
+                      const int64_t* rows, int64_t nrows, double* out, int nthreads) {
+    att_job j;
+    memset(&j, 0, sizeof(j));
+    j.kind = 1;
+    j.q = q; j.k = k; j.v = v;
+    j.cu = cu; j.B = B; j.H = H; j.D = D;
+    j.ds_q = 1.0; j.ds_k = 1.0; j.ds_v = 1.0; j.scale = scale;
+    j.pquant = 0; j.lrule = 0;
+    j.rows = rows; j.nrows = nrows; j.out = out;
+    return run_attention(&j, nthreads);
+}

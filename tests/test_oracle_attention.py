@@ -1,0 +1,154 @@
+"""Pins for the oracle's fp64 attention (CPU only).
+
+vLLM-Omni docs, "Quantized KV Cache", overview: Q/K/V are quantised
+dynamically right before the (full, non-causal) attention operator.  The
+pages give no numeric attention outputs, so the oracle is pinned by a
+library special case (softmax from scipy with no P quantisation), closed
+forms (Q = 0, a single key, hand-worked two-key cases that exercise the
+e4m3(256 p) rule), and invariants.
+"""
+import math
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle
+import synthetic
+
+
+def _codes(shape, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(*shape, generator=g) * scale
+    return x.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def _decode_torch(codes):
+    return torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def _softmax_attention(q, k, v, cu, scale):
+    """Library special case: per sequence and head, softmax(q k^T s) v."""
+    T, H, D = q.shape
+    out = np.empty((T, H, D))
+    for b in range(len(cu) - 1):
+        s0, s1 = cu[b], cu[b + 1]
+        for h in range(H):
+            S = q[s0:s1, h] @ k[s0:s1, h].T * scale
+            out[s0:s1, h] = scipy.special.softmax(S, axis=-1) @ v[s0:s1, h]
+    return out
+
+
+@pytest.mark.parametrize("lens", [[1, 5, 16], [8], [3, 3]])
+def test_unquantized_p_matches_library_softmax(lens):
+    H, D = 2, 128
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(cu[-1])
+    q8, k8, v8 = (_codes((T, H, D), s, 2.0) for s in (1, 2, 3))
+    ds = (0.031, 0.07, 1.7)
+    scale = 1.0 / math.sqrt(D)
+    got = oracle.attention_fp8(q8, k8, v8, cu, ds, pquant=False)
+    want = _softmax_attention(_decode_torch(q8) * ds[0], _decode_torch(k8) * ds[1],
+                              _decode_torch(v8) * ds[2], cu, scale)
+    np.testing.assert_allclose(got, want, rtol=1e-11, atol=1e-13)
+
+
+def test_bf16_attention_matches_library_softmax():
+    q, k, v, cu = synthetic.small_qkv(9, [4, 13], H=2, D=128)
+    got = oracle.attention_bf16(synthetic.bf16_bits(q), synthetic.bf16_bits(k),
+                                synthetic.bf16_bits(v), cu)
+    f = lambda t: t.to(torch.float64).numpy()
+    want = _softmax_attention(f(q), f(k), f(v), cu, 1.0 / math.sqrt(128))
+    np.testing.assert_allclose(got, want, rtol=1e-11, atol=1e-13)
+
+
+def test_zero_query_gives_mean_of_v_exactly_even_with_pquant():
+    # every score is 0, so p = 1, 256 p = 256 is an E4M3 value, p~ = 1
+    T, H, D = 37, 2, 128
+    cu = np.array([0, T], dtype=np.int32)
+    q8 = np.zeros((T, H, D), np.uint8)
+    k8, v8 = _codes((T, H, D), 4), _codes((T, H, D), 5)
+    ds_v = 0.75
+    got = oracle.attention_fp8(q8, k8, v8, cu, (0.5, 0.5, ds_v), pquant=True)
+    mean_v = _decode_torch(v8).mean(axis=0) * ds_v
+    for t in range(T):
+        np.testing.assert_allclose(got[t], mean_v, rtol=1e-14, atol=1e-15)
+
+
+def test_single_key_returns_that_value():
+    H, D = 3, 128
+    cu = np.array([0, 1, 2], dtype=np.int32)        # two sequences of length 1
+    q8, k8, v8 = (_codes((2, H, D), s, 3.0) for s in (6, 7, 8))
+    got = oracle.attention_fp8(q8, k8, v8, cu, (1.3, 0.2, 0.4), pquant=True)
+    np.testing.assert_array_equal(got, _decode_torch(v8) * 0.4)
+
+
+def _two_key_case(s1_code):
+    """q = e_0, k0 = 0, k1 = value(s1_code) e_0, v0 = 0, v1 = e_1; unit scales."""
+    D = 128
+    q8 = np.zeros((2, 1, D), np.uint8)
+    k8 = np.zeros((2, 1, D), np.uint8)
+    v8 = np.zeros((2, 1, D), np.uint8)
+    q8[:, 0, 0] = 0x38            # 1.0
+    k8[1, 0, 0] = s1_code
+    v8[1, 0, 1] = 0x38            # v1 = e_1
+    cu = np.array([0, 2], dtype=np.int32)
+    return q8, k8, v8, cu
+
+
+def test_pquant_rule_normal_range():
+    # s = (0, -0.125): p1 = e^-0.125 = 0.88250; 256 p1 = 225.92 lies in
+    # [128, 256) where E4M3 spacing is 16, nearest 224 -> p~1 = 0.875.
+    # l is the unquantised sum 1 + e^-0.125.
+    q8, k8, v8, cu = _two_key_case(0xA0)      # 0xA0 = -0.125
+    o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True)
+    want = 0.875 / (1.0 + math.exp(-0.125))
+    assert abs(o[0, 0, 1] - want) < 1e-15
+    assert o[0, 0, 0] == 0.0
+    # the unquantised and the "l = sum p~" variants differ visibly
+    o_none = oracle.attention_fp8(q8, k8, v8, cu, (1, 1, 1), scale=1.0, pquant=False)
+    assert abs(o_none[0, 0, 1] - math.exp(-0.125) / (1 + math.exp(-0.125))) < 1e-15
+    o_lq = oracle.attention_fp8(q8, k8, v8, cu, (1, 1, 1), scale=1.0, pquant=True,
+                                l_of_quantized=True)
+    assert abs(o_lq[0, 0, 1] - 0.875 / 1.875) < 1e-15
+
+
+def test_pquant_rule_subnormal_range():
+    # s = (0, -12): p1 = e^-12 = 6.144e-6; 256 p1 = 1.573e-3 is below 2^-6,
+    # in the subnormal range with spacing 2^-9 = 1.953e-3, so it rounds to
+    # 2^-9 and p~1 = 2^-9 / 256 = 2^-17.
+    q8, k8, v8, cu = _two_key_case(0xD4)      # 0xD4 = -12.0
+    o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True)
+    want = 2.0 ** -17 / (1.0 + math.exp(-12.0))
+    assert abs(o[0, 0, 1] - want) < 1e-20
+
+
+def test_rows_sum_to_one_and_columns_stay_in_range():
+    H, D = 2, 128
+    lens = [40, 7]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(cu[-1])
+    q8, k8, v8 = (_codes((T, H, D), s, 4.0) for s in (10, 11, 12))
+    ones = np.full((T, H, D), 0x38, np.uint8)
+    o = oracle.attention_fp8(q8, k8, ones, cu, (0.3, 0.3, 1.0), pquant=False)
+    np.testing.assert_allclose(o, 1.0, rtol=0, atol=1e-14)
+    oq = oracle.attention_fp8(q8, k8, ones, cu, (0.3, 0.3, 1.0), pquant=True)
+    # |p~ - p| <= p / 16 for normal codes; subnormal p~ adds at most 2^-18 each
+    assert np.all(np.abs(oq - 1.0) <= 2.0 ** -4 + 64 * 2.0 ** -17)
+    o = oracle.attention_fp8(q8, k8, v8, cu, (0.3, 0.3, 1.0), pquant=False)
+    vv = _decode_torch(v8)
+    for b in range(len(lens)):
+        sl = slice(cu[b], cu[b + 1])
+        lo, hi = vv[sl].min(axis=0), vv[sl].max(axis=0)
+        assert np.all(o[sl] >= lo - 1e-12) and np.all(o[sl] <= hi + 1e-12)
+
+
+def test_row_subset_equals_full_rows():
+    H, D = 2, 128
+    cu = np.array([0, 20, 33], dtype=np.int32)
+    q8, k8, v8 = (_codes((33, H, D), s, 2.0) for s in (13, 14, 15))
+    full = oracle.attention_fp8(q8, k8, v8, cu, (0.1, 0.2, 0.3))
+    rows = [0, 19, 20, 32, 5]
+    sub = oracle.attention_fp8(q8, k8, v8, cu, (0.1, 0.2, 0.3), rows=rows)
+    np.testing.assert_array_equal(sub, full[rows])
