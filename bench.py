@@ -1,0 +1,433 @@
+#!/usr/bin/env python
+"""Benchmark of the FP8 attention hot path on B200.
+
+One step = one pass of the path over the kernel-level workload of the vLLM
+FP8 ViT page's performance section (head_dim 128, seq_len 8192): 1 sequence,
+S=8192, 16 heads, bf16 Q/K/V ~ N(0,1) (synthetic), static per-tensor scales
+q=224, k=198, v=210 (the page's scale-file example):
+    fused quantise (static) -> varlen FP8 attention forward.
+Metric: attention TFLOP/s counted as 4 S^2 D H per step (5.498e11), plus the
+attention kernel's microseconds and the fused quantise kernel's GB/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun, one rank per GPU, each rank its own independent
+copy of the workload (weak scaling, no collective on the data path); the
+reported time is the max over ranks.  ``--impl reference`` times the CPU
+oracle on the host cores on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+S, H, D = 8192, 16, 128
+STATIC = (224.0, 198.0, 210.0)
+FLOPS_PER_STEP = 4.0 * S * S * D * H                  # 5.498e11
+QUANT_BYTES_PER_STEP = 3.0 * S * H * D * 3            # 2 B read + 1 B write per element
+METRIC = "FP8 attn fwd TFLOP/s (4·S²·D·H) & µs @S=8192 D=128; fused quant GB/s"
+WORKLOAD = "kernel_s8192_h16_d128_static_224_198_210"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_PER_BF16 = 2.0                                    # nominal dense ratio (4.5 / 2.25 PF)
+ATTN_SOURCES = ["quantization_amax_reduce_b200/csrc/attention.cu",
+                "quantization_amax_reduce_b200/csrc/sm100_ptx.cuh"]
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_fp8_s8192_h16.md")
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=50)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--e2e-steps", type=int, default=0,
+                   help="steps of the host-buffer end-to-end leg (default: steps/20, >= 5)")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------
+# helpers shared with the multi-process tests
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(value: float, dist=None, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity without a group)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(units_per_rank: float, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: the units every rank processed / the slowest rank's time."""
+    return units_per_rank * world / max_seconds
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_digest(paths) -> str:
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, or None
+    when the kernel sources changed since it was captured."""
+    if not os.path.exists(PROFILE_SUMMARY):
+        return None
+    vals = {}
+    with open(PROFILE_SUMMARY) as f:
+        for line in f:
+            if ":" in line and line.strip().startswith("- "):
+                k, v = line.strip()[2:].split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    try:
+        if vals.get("source_digest") != source_digest(ATTN_SOURCES):
+            return None
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.seek(0)
+        rows = [r.split(",") for r in self.out.read().strip().splitlines() if r.strip()]
+        self.out.close()
+        os.unlink(self.out.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 8:
+                continue
+            try:
+                sm.append(float(r[0]))
+                mx = float(r[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, r[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(n_rows: int, quant_tokens: int, seed: int = 0):
+    """Time the oracle on a bounded sample of the workload: static quantise of
+    `quant_tokens` tokens of Q/K/V and fp64 attention for `n_rows` query rows
+    of every head over all S keys.  Returns (seconds, attention FLOPs of the
+    sample, quantised elements, threads)."""
+    import numpy as np
+    import oracle
+    import synthetic
+    q, k, v, cu = synthetic.qkv(3)
+    sub_cu = np.array([0, quant_tokens], dtype=np.int32)
+    bits = [synthetic.bf16_bits(x[:quant_tokens]) for x in (q, k, v)]
+    full_bits = [synthetic.bf16_bits(x) for x in (q, k, v)]
+    rng = np.random.Generator(np.random.PCG64(seed))
+    rows = np.sort(rng.choice(S, size=n_rows, replace=False))
+    threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    codes = []
+    for x, A in zip(bits, STATIC):
+        qs, ds = oracle.scales_from_bound(A)
+        codes.append(oracle.quantize(x, sub_cu, H, D, qs))
+    t1 = time.perf_counter()
+    # attention needs the codes of all keys: quantise the rest outside the clock
+    full = []
+    for x, A in zip(full_bits, STATIC):
+        qs, ds = oracle.scales_from_bound(A)
+        full.append(oracle.quantize(x, cu, H, D, qs))
+    dsv = [float(oracle.scales_from_bound(A)[1]) for A in STATIC]
+    t2 = time.perf_counter()
+    oracle.attention_fp8(*full, cu, dsv, rows=rows)
+    t3 = time.perf_counter()
+    return (t1 - t0) + (t3 - t2), 4.0 * n_rows * S * D * H, 3 * quant_tokens * H * D, threads
+
+
+def cpu_baseline_full_step_estimate():
+    """Oracle time for one full step, from a bounded sample: full quantisation
+    of Q/K/V plus attention for 32 of the 8192 query rows (x256)."""
+    import numpy as np
+    import oracle
+    import synthetic
+    q, k, v, cu = synthetic.qkv(3)
+    threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    codes = []
+    for x, A in zip((q, k, v), STATIC):
+        qs, _ = oracle.scales_from_bound(A)
+        codes.append(oracle.quantize(synthetic.bf16_bits(x), cu, H, D, qs))
+    t1 = time.perf_counter()
+    dsv = [float(oracle.scales_from_bound(A)[1]) for A in STATIC]
+    n_rows = 32
+    rows = np.sort(np.random.Generator(np.random.PCG64(1)).choice(S, size=n_rows, replace=False))
+    oracle.attention_fp8(*codes, cu, dsv, rows=rows)
+    t2 = time.perf_counter()
+    step_s = (t1 - t0) + (t2 - t1) * (S / n_rows)
+    return {
+        "value": FLOPS_PER_STEP / step_s / 1e12,
+        "unit": "TFLOP/s",
+        "cores": threads,
+        "kind": "oracle",
+        "sample": (f"full static quantisation of Q/K/V ({t1 - t0:.2f} s) + fp64 attention of "
+                   f"{n_rows}/{S} query rows x {H} heads ({t2 - t1:.2f} s, scaled x{S // n_rows})"),
+        "seconds_per_step": step_s,
+    }
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    total = args.steps + args.warmup
+    # size each step so the whole run takes about two minutes
+    t_probe, f_probe, _, threads = oracle_sample(2, 256)
+    per_row = max(t_probe / 2, 1e-4)
+    budget = 120.0 / max(total, 1)
+    n_rows = int(max(1, min(512, budget / per_row)))
+    quant_tokens = max(16, min(S, n_rows * 16))
+    for _ in range(args.warmup):
+        oracle_sample(n_rows, quant_tokens)
+    secs, flops = 0.0, 0.0
+    for i in range(args.steps):
+        s, f, _, threads = oracle_sample(n_rows, quant_tokens, seed=i)
+        secs += s
+        flops += f
+    value = flops / secs / 1e12
+    sample = (f"per step: oracle static quantisation of {quant_tokens} tokens of Q/K/V and fp64 "
+              f"attention of {n_rows} query rows x {H} heads over all {S} keys")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "S": S, "heads": H, "head_dim": D},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import synthetic
+    import quantization_amax_reduce_b200 as qar
+
+    rank, world, local_rank = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    # inputs resident in HBM; each rank its own draw (layer index = rank)
+    q, k, v, cu = synthetic.qkv(3, layer=rank, device=dev)
+    cu_d = torch.as_tensor(cu, device=dev)
+    ctx = qar.Context(1, device=dev)
+    ctx.set_static_scales(0, *STATIC)
+    q8, k8, v8 = (torch.empty((S, H, D), dtype=torch.uint8, device=dev) for _ in range(3))
+    out = torch.empty((S, H, D), dtype=torch.bfloat16, device=dev)
+    ds_ptr = ctx.descale_ptr(0)
+    stream = torch.cuda.current_stream(dev)
+
+    def quant():
+        ctx.quantize_qkv(0, qar.STATIC, q, k, v, cu_d, S, out=(q8, k8, v8), stream=stream)
+
+    def attn():
+        qar.varlen_fwd(q8, k8, v8, cu_d, S, ds_ptr, out=out, stream=stream)
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
+    for _ in range(args.warmup):
+        quant()
+        attn()
+    torch.cuda.synchronize(dev)
+    if ctx.get_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    uuid = getattr(torch.cuda.get_device_properties(dev), "uuid", None)
+    sampler = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(local_rank))
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    launches0 = qar.launch_count()
+    wall0 = time.perf_counter()
+    for i in range(K):
+        flush.zero_()                       # L2 flushed between timed steps
+        ev[i][0].record(stream)
+        quant()
+        ev[i][1].record(stream)
+        attn()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    wall = time.perf_counter() - wall0
+    launches = qar.launch_count() - launches0
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+    clocks = sampler.stop()
+    quant_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    attn_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    total_s = (sum(quant_ms) + sum(attn_ms)) / 1e3
+    max_total_s = max_over_ranks(total_s, dist if world > 1 else None, dev)
+    if ctx.get_error() != 0:
+        raise RuntimeError("device error during the timed region")
+
+    # end to end through the public API with pinned host buffers
+    E = args.e2e_steps or max(5, K // 20)
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    hout = torch.empty((S, H, D), dtype=torch.bfloat16).pin_memory()
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(E + 2)]
+    for i in range(E + 2):
+        if i >= 2:
+            flush.zero_()
+            e2e_ev[i][0].record(stream)
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        quant()
+        attn()
+        hout.copy_(out, non_blocking=True)
+        if i >= 2:
+            e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_s = sum(e2e_ev[i][0].elapsed_time(e2e_ev[i][1]) for i in range(2, E + 2)) / 1e3
+    e2e_max = max_over_ranks(e2e_s, dist if world > 1 else None, dev)
+
+    result = None
+    if rank == 0:
+        peaks, src = load_peaks()
+        fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
+        attn_s = statistics.mean(attn_ms) / 1e3
+        quant_s = statistics.mean(quant_ms) / 1e3
+        attn_tflops = FLOPS_PER_STEP / attn_s / 1e12
+        quant_gbs = QUANT_BYTES_PER_STEP / quant_s / 1e9
+        value = aggregate_throughput(FLOPS_PER_STEP * K, world, max_total_s) / 1e12
+        share_attn = sum(attn_ms) / (sum(attn_ms) + sum(quant_ms))
+        result = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": max_total_s / K * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "S": S, "heads": H, "head_dim": D, "batch": 1,
+                       "scales": "static q=224 k=198 v=210", "l2": "flushed between steps",
+                       "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"},
+            "attn_us": attn_s * 1e6, "attn_tflops": attn_tflops,
+            "quant_us": quant_s * 1e6, "quant_gbs": quant_gbs,
+            "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": fp8_peak,
+                         "unit": "TFLOP/s", "frac": attn_tflops / fp8_peak,
+                         "traffic": profiled_traffic(),
+                         "kernel": "attn_fwd_kernel<fp8>",
+                         "peak_source": f"{src} bf16 burst x{FP8_PER_BF16:g} (fp8/bf16 nominal)"},
+            "quant_roofline": {"bound": "hbm", "achieved": quant_gbs, "peak": peaks["hbm_gbs"],
+                               "unit": "GB/s", "frac": quant_gbs / peaks["hbm_gbs"],
+                               "kernel": "quant_static_kernel", "peak_source": src},
+            "kernel_share": {"attn_fwd_kernel<fp8>": share_attn,
+                             "quant_static_kernel": 1.0 - share_attn},
+            "e2e": {"value": FLOPS_PER_STEP * E * world / e2e_max / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": 3 * S * H * D * 2, "d2h_bytes_per_step": S * H * D * 2,
+                    "steps": E},
+            "gpu_launches": launches,
+            "wall_s_timed": wall,
+        }
+        if clocks is not None:
+            result["clocks"] = clocks
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+        dist.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline_full_step_estimate()
+        print(json.dumps(result))
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,239 @@
+/*
+ * fp8attn -- on-the-fly FP8 (E4M3) quantisation of Q/K/V with per-tensor
+ * scales, followed by a varlen, non-causal FP8 flash-attention forward, for
+ * NVIDIA B200 (sm_100a).  Plain C ABI: device pointers are raw CUDA device
+ * addresses, host pointers are ordinary host memory, streams are
+ * `cudaStream_t` values passed as `void*` (NULL = the legacy default stream).
+ *
+ * Method (web pages on FP8 ViT / DiT attention):
+ *   - vLLM docs, "FP8 ViT encoder attention": Q/K/V are quantised to FP8 on
+ *     the fly right before the attention call (introduction); by default a
+ *     circular buffer of 16 observed Q/K/V amax values drives the per-forward
+ *     scale update (usage section); static per-layer scales can be calibrated
+ *     once -- 16 dynamic passes, then the learned scales are saved multiplied
+ *     by a save margin, default 1.5 -- and reused (usage section, scale file
+ *     format section); the reference cost is three quantisation launches plus
+ *     an unpadding step (notes).
+ *   - vLLM-Omni docs, "Quantized KV Cache": eligible full (non-causal)
+ *     attention forwards use FP8; layers named by a selector of
+ *     comma-separated integers and inclusive ranges keep the native dtype
+ *     (parameters table).
+ *   - Ascend quantisation chapter: FP8 formats E4M3 / E5M2 (names only).
+ *
+ * Readings where the pages are silent (each is fixed here):
+ *   - E4M3 is the OCP "FN" format: max 448, no infinities; casts round to
+ *     nearest even and saturate to +-448; NaN casts to 0x7F.
+ *   - amax = max |x| over the valid (unpadded) tokens of one tensor; NaN is
+ *     ignored; an infinite amax is reported (FP8ATTN_ERR_NONFINITE) and not
+ *     pushed.
+ *   - Dynamic scaling is current-inclusive: the pass's amax is pushed into
+ *     the 16-entry ring first, then A = max over the filled slots.
+ *   - qs = fl32(448 / A), ds = fl32(A / 448) (each one correctly rounded fp32
+ *     division); A == 0 gives qs = ds = 1.  code = e4m3(fl32(x * qs)).
+ *   - Static values are bounds A in activation units with the margin already
+ *     applied (the margin multiplies saved values once, at export).
+ *   - Attention: s = q8.k8 * ds_q * ds_k * softmax_scale; p = exp(s - m)
+ *     with m the running row max; P for the PV product is e4m3(256 p); the
+ *     row sum l accumulates the unquantised p; out = bf16(O * ds_v / (256 l)).
+ *
+ * Layouts: bf16 sources are addressed as (token, head, channel) with the
+ * channel contiguous (head_dim == 128) and element strides `tok_stride`,
+ * `head_stride` (multiples of 8; 16-byte aligned base), so packed [T,H,D],
+ * padded [B,S_max,H,D] and interleaved [T,3,H,D] sources all work.  FP8
+ * outputs and attention inputs/outputs are packed [T,H,D] with
+ * T = total_tokens (the row count of those buffers).
+ *
+ * Errors: host-detectable problems return a status at once and launch
+ * nothing.  Problems found on the device (inconsistent cu_seqlens, a wait
+ * that ran past its time limit, a non-finite amax) set a device error word
+ * and the kernel skips the affected work without trapping;
+ * fp8attn_get_error() reports and clears it.
+ *
+ * Ownership: the caller allocates and owns every buffer, including the
+ * context's device workspace; a context owns only a small host struct.
+ * All launches are asynchronous on the given stream; functions that read
+ * results back to the host synchronise that stream and say so.
+ */
+#ifndef FP8ATTN_H_
+#define FP8ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FP8ATTN_OK = 0,
+  FP8ATTN_ERR_INVALID = 1,     /* bad argument (null, negative, out of range) */
+  FP8ATTN_ERR_CUDA = 2,        /* a CUDA runtime / driver call failed */
+  FP8ATTN_ERR_TIMEOUT = 3,     /* a device-side wait gave up (work skipped) */
+  FP8ATTN_ERR_UNSUPPORTED = 4, /* valid but unsupported (head_dim != 128, ...) */
+  FP8ATTN_ERR_NONFINITE = 5,   /* an observed amax was infinite (not pushed) */
+  FP8ATTN_ERR_SEQLENS = 6      /* cu_seqlens inconsistent with batch/max_seqlen */
+} fp8attn_status;
+
+/* Per-layer quantisation mode (host-side selection). */
+typedef enum {
+  FP8ATTN_DYNAMIC = 0, /* amax ring, current pass included */
+  FP8ATTN_STATIC = 1,  /* static bounds set by fp8attn_set_static_scales */
+  FP8ATTN_SKIP = 2     /* native bf16 attention, no quantisation */
+} fp8attn_mode;
+
+typedef struct fp8attn_ctx fp8attn_ctx;
+
+/* Human-readable name of a status code (static string). */
+const char* fp8attn_status_string(int status);
+
+/* Entries per amax ring: 16 (vLLM FP8 ViT page, usage section). */
+int fp8attn_ring_length(void);
+
+/* Bytes of device workspace a context for `num_layers` layers needs (ring,
+ * scales, static bounds, grid-barrier words, error word). 0 if num_layers<1. */
+size_t fp8attn_workspace_bytes(int num_layers);
+
+/* Create a context over caller-owned device workspace `d_workspace` of at
+ * least fp8attn_workspace_bytes(num_layers) bytes (256-byte aligned).  The
+ * workspace is zeroed on `stream` (empty rings, no static scales).  The
+ * current CUDA device must be the workspace's device.  *out receives the
+ * context.  Errors: INVALID (null pointers, too small, misaligned), CUDA. */
+fp8attn_status fp8attn_create(int num_layers, void* d_workspace, size_t workspace_bytes,
+                              void* stream, fp8attn_ctx** out);
+
+/* Free the host struct (the workspace stays the caller's). */
+fp8attn_status fp8attn_destroy(fp8attn_ctx* ctx);
+
+/* Fused amax-reduce + ring/scale update + E4M3 cast + unpad of Q, K and V
+ * for one layer, in a single launch (replaces the pages' three quantisation
+ * launches plus unpadding).
+ *   mode DYNAMIC: amax of each tensor over its valid tokens; push into the
+ *     layer's ring; A = ring max; cast with qs = 448/A.  STATIC: cast with the
+ *     layer's static bounds (error INVALID if none were set).  SKIP: INVALID.
+ *   q, k, v: bf16 sources; element (t_src, h, d) at base + t_src*tok_stride
+ *     + h*head_stride + d.  d_src_seq_start: NULL if the source is packed
+ *     (t_src = t); else int32[batch], the source row of each sequence's first
+ *     token (padded source).  d_cu_seqlens: int32[batch+1], non-decreasing,
+ *     cu[0] = 0, each length <= max_seqlen, cu[batch] == total_tokens.
+ *   q8, k8, v8: E4M3 outputs, packed [total_tokens, num_heads, head_dim].
+ * The layer's scales (fp8attn_descale_ptr) are updated on the device.
+ * Errors: INVALID, UNSUPPORTED (head_dim != 128, misaligned strides), CUDA;
+ * device-side: SEQLENS (nothing written), NONFINITE, TIMEOUT. */
+fp8attn_status fp8attn_quantize_qkv(fp8attn_ctx* ctx, int layer, int mode, const void* q,
+                                    const void* k, const void* v, int64_t tok_stride,
+                                    int64_t head_stride, const int32_t* d_src_seq_start,
+                                    const int32_t* d_cu_seqlens, int batch, int max_seqlen,
+                                    int64_t total_tokens, int num_heads, int head_dim, void* q8,
+                                    void* k8, void* v8, void* stream);
+
+/* Push three externally observed amax values (device float[3]: q, k, v) into
+ * the layer's rings and recompute its scales, on the device (vLLM FP8 ViT
+ * page, usage section: the ring drives the per-forward scale).  A NaN or
+ * infinite value is not pushed and sets NONFINITE.  Errors: INVALID, CUDA. */
+fp8attn_status fp8attn_amax_ring_update(fp8attn_ctx* ctx, int layer, const float* d_amax3,
+                                        void* stream);
+
+/* Set a layer's static bounds (values as stored in a scale file: q, k, v,
+ * margin already applied; vLLM FP8 ViT page, scale file format section).
+ * Enqueues a small host->device copy on `stream`.  Errors: INVALID
+ * (negative or non-finite value, bad layer), CUDA. */
+fp8attn_status fp8attn_set_static_scales(fp8attn_ctx* ctx, int layer, float q, float k,
+                                         float v, void* stream);
+
+/* Forget a layer's static bounds (host-side flag only). */
+fp8attn_status fp8attn_clear_static_scales(fp8attn_ctx* ctx, int layer);
+
+/* 1 if the layer has static bounds, 0 if not, -1 on a bad argument. */
+int fp8attn_has_static_scales(const fp8attn_ctx* ctx, int layer);
+
+/* Export the calibrated static values for every layer: h_out[l*3 + t] =
+ * fl32(max(ring of tensor t of layer l) * margin), t = q, k, v (vLLM FP8 ViT
+ * page, usage section: saved scales are multiplied by the save margin,
+ * default 1.5).  Synchronises `stream`.  Errors: INVALID, CUDA. */
+fp8attn_status fp8attn_export_static_scales(fp8attn_ctx* ctx, float margin, float* h_out,
+                                            void* stream);
+
+/* Device pointer to the layer's current descales {ds_q, ds_k, ds_v} (fp32),
+ * as written by the last quantisation of that layer -- the scale argument of
+ * fp8attn_varlen_fwd.  NULL on a bad argument. */
+const float* fp8attn_descale_ptr(fp8attn_ctx* ctx, int layer);
+
+/* Device pointer to the layer's current quantisation scales {qs_q, qs_k, qs_v}. */
+const float* fp8attn_quant_scale_ptr(fp8attn_ctx* ctx, int layer);
+
+/* Copy the layer's ring state to the host: h_slots float[3][16],
+ * h_meta uint32[3][2] = {head, count} per tensor.  Synchronises `stream`. */
+fp8attn_status fp8attn_get_ring_state(fp8attn_ctx* ctx, int layer, float* h_slots,
+                                      uint32_t* h_meta, void* stream);
+
+/* Restore a ring state saved by fp8attn_get_ring_state (resume) and
+ * recompute the layer's dynamic scales from it.  Synchronises `stream`. */
+fp8attn_status fp8attn_set_ring_state(fp8attn_ctx* ctx, int layer, const float* h_slots,
+                                      const uint32_t* h_meta, void* stream);
+
+/* Copy the layer's current {qs_q, qs_k, qs_v, ds_q, ds_k, ds_v} to the host.
+ * Synchronises `stream`. */
+fp8attn_status fp8attn_get_scales(fp8attn_ctx* ctx, int layer, float* h_out6, void* stream);
+
+/* Varlen, non-causal FP8 attention forward (vLLM-Omni "Quantized KV Cache"
+ * overview: the quantised Q/K/V feed the attention operator; vLLM FP8 ViT
+ * page: per-tensor scales).  q8, k8, v8: E4M3 packed [T, num_heads, 128]
+ * with T = total_tokens (the buffers' row count; the kernel never reads past
+ * it); d_cu_seqlens int32[batch+1] with cu[batch] <= T; d_descale_qkv: device float[3] {ds_q, ds_k,
+ * ds_v}; softmax_scale: 0 selects 1/sqrt(head_dim); out: bf16 [T, num_heads,
+ * 128].  Each token attends to every token of its own sequence.  The base
+ * pointers must be 16-byte aligned.  d_error: optional device int32 that
+ * receives FP8ATTN_ERR_SEQLENS / FP8ATTN_ERR_TIMEOUT bits (may be NULL).
+ * Errors: INVALID, UNSUPPORTED (head_dim != 128), CUDA. */
+fp8attn_status fp8attn_varlen_fwd(const void* q8, const void* k8, const void* v8,
+                                  const int32_t* d_cu_seqlens, int batch, int max_seqlen,
+                                  int64_t total_tokens, int num_heads, int head_dim,
+                                  const float* d_descale_qkv,
+                                  float softmax_scale, void* out, int32_t* d_error,
+                                  void* stream);
+
+/* Native-dtype attention for skipped layers (vLLM-Omni "Quantized KV Cache",
+ * parameters table: selected layers keep the native dtype): the same
+ * computation on bf16 q, k, v [T, num_heads, 128] with no quantisation. */
+fp8attn_status fp8attn_varlen_fwd_bf16(const void* q, const void* k, const void* v,
+                                       const int32_t* d_cu_seqlens, int batch, int max_seqlen,
+                                       int64_t total_tokens, int num_heads, int head_dim,
+                                       float softmax_scale,
+                                       void* out, int32_t* d_error, void* stream);
+
+/* Read and clear the context's device error word (synchronises `stream`).
+ * Returns OK or the most severe device-side status seen since the last call.
+ * After a TIMEOUT the context's grid-barrier words are reset. */
+fp8attn_status fp8attn_get_error(fp8attn_ctx* ctx, void* stream);
+
+/* Read and clear a caller-owned device error word as filled by
+ * fp8attn_varlen_fwd (synchronises `stream`). */
+fp8attn_status fp8attn_read_error_word(int32_t* d_error, void* stream);
+
+/* Parse a layer/step selector: comma-separated non-negative integers and
+ * inclusive ranges "a-b" (vLLM-Omni "Quantized KV Cache", parameters table,
+ * e.g. "0,1,4-6" and "0-2,10").  Spaces around items are allowed; NULL or
+ * an empty string selects nothing.  mask_out: uint8[max_index], set to 1 for
+ * selected indices, 0 otherwise.  Errors: INVALID for malformed items,
+ * reversed ranges or indices >= max_index (mask_out then all zero). */
+fp8attn_status fp8attn_parse_selector(const char* text, int max_index, uint8_t* mask_out);
+
+/* Mode of a layer: SKIP if skip_mask[layer] (skip_mask may be NULL),
+ * else STATIC if the context has static bounds for it, else DYNAMIC.
+ * -1 on a bad argument. */
+int fp8attn_select_mode(const fp8attn_ctx* ctx, const uint8_t* skip_mask, int layer);
+
+/* E4M3 cast helper: d_out[i] = e4m3(fl32(d_in[i] * scale)), fp32 device
+ * input, n elements, the same conversion the quantisation kernel uses. */
+fp8attn_status fp8attn_e4m3_encode(const float* d_in, int64_t n, float scale, void* d_out,
+                                   void* stream);
+
+/* Number of kernels the library has launched in this process (a counter
+ * incremented on every successful launch; for accounting in benchmarks). */
+uint64_t fp8attn_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8ATTN_H_ */

@@ -32,6 +32,7 @@ RING_LEN = 16          # vLLM FP8 ViT page: 16 observed amax values
 DEFAULT_MARGIN = 1.5   # vLLM FP8 ViT page: --mm-encoder-fp8-scale-save-margin
 E4M3_MAX = 448.0       # OCP E4M3 (FN) largest finite magnitude
 P_SCALE = 256.0        # P is quantised as e4m3(256 p) (power of two: exact)
+P_BLOCK = 128          # keys per P-quantisation block (running-max reference)
 
 
 class _Ring(ctypes.Structure):
@@ -227,9 +228,10 @@ def attention_fp8(q8, k8, v8, cu, ds_qkv: Sequence[float], scale: Optional[float
                   nthreads: int = 0) -> np.ndarray:
     """fp64 attention on E4M3 codes [T, H, D]; returns [len(rows) or T, H, D].
 
-    p = exp(s - M) with M the row's final max; the PV product uses
-    e4m3(256 p)/256 when ``pquant``; l is the sum of the unquantised p unless
-    ``l_of_quantized``."""
+    With ``pquant`` the PV product uses P quantised per block of 128 keys (in
+    sequence order) as e4m3(256 exp(s - m))/256, m the running row max over
+    the keys seen so far, carried exactly to the final max M; l is the sum of
+    the unquantised exp(s - M) unless ``l_of_quantized``."""
     q8 = np.ascontiguousarray(q8, dtype=np.uint8)
     k8 = np.ascontiguousarray(k8, dtype=np.uint8)
     v8 = np.ascontiguousarray(v8, dtype=np.uint8)

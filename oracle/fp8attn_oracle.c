@@ -28,9 +28,12 @@
  *     ds = fl32(A/448); A == 0 gives qs = ds = 1.
  *   - static values are bounds A in activation units (the margin is applied
  *     when they are saved, never again on load).
- *   - attention quantises p = exp(s - M) (M = the row's final max) as
- *     e4m3(256 p)/256 for the PV product and normalises by l = sum of the
- *     unquantised p.
+ *   - attention: P for the PV product is quantised block by block (128
+ *     keys, in sequence order) as e4m3(256 exp(s - m))/256 against the
+ *     running row max m over the keys seen so far -- the rule a single-pass
+ *     (online-softmax) kernel applies -- and carried to the final max M
+ *     exactly; the output is normalised by l = sum of the unquantised
+ *     exp(s - M).
  *
  * Floating point: quantisation follows the kernel's stated fp32 rules (one
  * fp32 RN multiply, one fp32 RN division), attention is evaluated in fp64.
@@ -339,11 +342,18 @@ static double elem(const att_job* j, const void* base, int64_t t, int h, int d) 
     return (double)bf16_to_f32(((const uint16_t*)base)[idx]);
 }
 
+/* P rule: the PV product takes P in blocks of OR_P_BLOCK keys, visited in
+ * order from the start of the sequence; each block's p are quantised as
+ * e4m3(256 exp(s - m_t)) / 256 against the running max m_t over the keys
+ * seen so far (blocks 0..t), then carried to the final max M by the exact
+ * factor exp(m_t - M).  l is the sum of the unquantised p = exp(s - M). */
+#define OR_P_BLOCK 128
+
 static void attend_one(const att_job* j, int64_t ri, int h, double* s_buf) {
     int64_t t = j->rows ? j->rows[ri] : ri;
     int b, d;
     int64_t k0, k1, kk;
-    double M = -INFINITY, l = 0.0;
+    double M = -INFINITY, l = 0.0, m_blk = -INFINITY;
     double* o = j->out + (ri * j->H + h) * (int64_t)j->D;
     double dsq = j->kind == 0 ? j->ds_q : 1.0;
     double dsk = j->kind == 0 ? j->ds_k : 1.0;
@@ -361,9 +371,18 @@ static void attend_one(const att_job* j, int64_t ri, int h, double* s_buf) {
     }
     for (d = 0; d < j->D; ++d) o[d] = 0.0;
     for (kk = k0; kk < k1; ++kk) {
-        double p = exp(s_buf[kk - k0] - M);
+        double s = s_buf[kk - k0];
+        double p = exp(s - M);
         double pt = p;
-        if (j->pquant) pt = or_e4m3_value(or_e4m3_encode(256.0 * p)) / 256.0;
+        if ((kk - k0) % OR_P_BLOCK == 0) {
+            /* entering a new block: running max over blocks seen so far */
+            int64_t e = kk + OR_P_BLOCK < k1 ? kk + OR_P_BLOCK : k1, x;
+            for (x = kk; x < e; ++x)
+                if (s_buf[x - k0] > m_blk) m_blk = s_buf[x - k0];
+        }
+        if (j->pquant)
+            pt = or_e4m3_value(or_e4m3_encode(256.0 * exp(s - m_blk))) / 256.0 *
+                 exp(m_blk - M);
         l += j->lrule ? pt : p;
         for (d = 0; d < j->D; ++d) o[d] += pt * elem(j, j->v, kk, h, d);
     }
@@ -406,8 +425,9 @@ static int run_attention(att_job* j, int nthreads) {
 }
 
 /* FP8 attention on E4M3 codes [T][H][D] with per-tensor descales.
- * o_i = (sum_j p~_ij dec(v_j)) * ds_v / l_i with p_ij = exp(s_ij - M_i),
- * s_ij = (sum_d dec(q_id) dec(k_jd)) * ds_q * ds_k * scale.
+ * o_i = (sum_j p~_ij dec(v_j)) * ds_v / l_i, l_i = sum_j exp(s_ij - M_i),
+ * s_ij = (sum_d dec(q_id) dec(k_jd)) * ds_q * ds_k * scale, and p~ by the
+ * block rule above.
  * Returns the number of threads used. */
 int or_attention_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
                      const int32_t* cu, int B, int H, int D,

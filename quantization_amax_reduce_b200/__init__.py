@@ -1,0 +1,408 @@
+"""fp8attn for B200 (sm_100a): on-the-fly FP8 (E4M3) quantisation of Q/K/V
+with per-tensor scales from a device-resident 16-entry amax ring or from
+static per-layer bounds, and a varlen non-causal FP8 flash-attention forward
+on tcgen05 tensor cores.
+
+This module is a thin ctypes binding over ``libfp8attn.so`` (built from
+``csrc/`` by ``build.py``): it only marshals torch tensors into device
+pointers, sizes and streams.  Every step of the path runs in the library's
+CUDA kernels; there is no CPU or PyTorch fallback, and every call fails
+loudly if the library is missing or no CUDA device is present.
+
+Names follow the C ABI in ``include/fp8attn.h`` without the ``fp8attn_``
+prefix.
+"""
+from __future__ import annotations
+
+import ctypes
+import json
+import math
+import os
+from typing import Dict, Iterable, List, Optional, Sequence, Tuple
+
+import numpy as np
+import torch
+
+__all__ = [
+    "DYNAMIC", "STATIC", "SKIP", "RING_LENGTH", "DEFAULT_MARGIN", "FP8AttnError", "lib",
+    "Context", "varlen_fwd", "varlen_fwd_bf16", "parse_selector", "e4m3_encode",
+    "launch_count", "load_scale_file", "save_scale_file", "read_error_word",
+]
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libfp8attn.so")
+
+DYNAMIC, STATIC, SKIP = 0, 1, 2
+RING_LENGTH = 16
+DEFAULT_MARGIN = 1.5
+HEAD_DIM = 128
+
+_STATUS = {
+    0: "ok", 1: "invalid argument", 2: "CUDA error", 3: "device wait timed out",
+    4: "unsupported configuration", 5: "non-finite amax", 6: "inconsistent cu_seqlens",
+}
+
+
+class FP8AttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_STATUS.get(status, 'status %d' % status)}")
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load ``libfp8attn.so`` (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m quantization_amax_reduce_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, I64, F, U8P = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
+                         ctypes.c_void_p)
+    sigs = {
+        "fp8attn_status_string": (ctypes.c_char_p, [I]),
+        "fp8attn_ring_length": (I, []),
+        "fp8attn_workspace_bytes": (ctypes.c_size_t, [I]),
+        "fp8attn_create": (I, [I, P, ctypes.c_size_t, P, ctypes.POINTER(P)]),
+        "fp8attn_destroy": (I, [P]),
+        "fp8attn_quantize_qkv": (I, [P, I, I, P, P, P, I64, I64, P, P, I, I, I64, I, I, P, P, P,
+                                     P]),
+        "fp8attn_amax_ring_update": (I, [P, I, P, P]),
+        "fp8attn_set_static_scales": (I, [P, I, F, F, F, P]),
+        "fp8attn_clear_static_scales": (I, [P, I]),
+        "fp8attn_has_static_scales": (I, [P, I]),
+        "fp8attn_export_static_scales": (I, [P, F, P, P]),
+        "fp8attn_descale_ptr": (P, [P, I]),
+        "fp8attn_quant_scale_ptr": (P, [P, I]),
+        "fp8attn_get_ring_state": (I, [P, I, P, P, P]),
+        "fp8attn_set_ring_state": (I, [P, I, P, P, P]),
+        "fp8attn_get_scales": (I, [P, I, P, P]),
+        "fp8attn_varlen_fwd": (I, [P, P, P, P, I, I, I64, I, I, P, F, P, P, P]),
+        "fp8attn_varlen_fwd_bf16": (I, [P, P, P, P, I, I, I64, I, I, F, P, P, P]),
+        "fp8attn_get_error": (I, [P, P]),
+        "fp8attn_read_error_word": (I, [P, P]),
+        "fp8attn_parse_selector": (I, [ctypes.c_char_p, I, U8P]),
+        "fp8attn_select_mode": (I, [P, U8P, I]),
+        "fp8attn_e4m3_encode": (I, [P, I64, F, P, P]),
+        "fp8attn_launch_count": (ctypes.c_uint64, []),
+    }
+    for name, (res, args) in sigs.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise FP8AttnError(status, what)
+
+
+def _require_cuda(t: torch.Tensor, name: str) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def _stream(stream, device) -> int:
+    if stream is None:
+        return torch.cuda.current_stream(device).cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _cu_tensor(cu, device) -> torch.Tensor:
+    if isinstance(cu, torch.Tensor):
+        if cu.dtype != torch.int32 or not cu.is_cuda:
+            raise ValueError("cu_seqlens must be an int32 CUDA tensor")
+        return cu
+    return torch.as_tensor(np.asarray(cu, dtype=np.int32), device=device)
+
+
+# ---------------------------------------------------------------------------
+# context: device-resident rings and scales
+# ---------------------------------------------------------------------------
+
+class Context:
+    """Per-model scale state (one amax ring + scales per attention layer).
+
+    The device workspace is a torch allocation owned by this object."""
+
+    def __init__(self, num_layers: int, device=None, stream=None):
+        L = lib()
+        self.device = torch.device(device if device is not None else "cuda")
+        if self.device.type != "cuda":
+            raise ValueError("Context needs a CUDA device")
+        self.num_layers = int(num_layers)
+        nbytes = L.fp8attn_workspace_bytes(self.num_layers)
+        if nbytes == 0:
+            raise ValueError("num_layers must be >= 1")
+        with torch.cuda.device(self.device):
+            self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+            h = ctypes.c_void_p()
+            _check(L.fp8attn_create(self.num_layers, _ptr(self.workspace), nbytes,
+                                    ctypes.c_void_p(_stream(stream, self.device)),
+                                    ctypes.byref(h)), "fp8attn_create")
+        self._h = h
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value and _lib is not None:
+            _lib.fp8attn_destroy(h)
+            self._h = None
+
+    # -- hot path ---------------------------------------------------------
+    def quantize_qkv(self, layer: int, mode: int, q: torch.Tensor, k: torch.Tensor,
+                     v: torch.Tensor, cu_seqlens, max_seqlen: int, *,
+                     total_tokens: Optional[int] = None, src_seq_start=None,
+                     out: Optional[Sequence[torch.Tensor]] = None, stream=None
+                     ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+        """Fused amax + ring/scale update + E4M3 cast + unpad of one layer's
+        Q, K, V.  Sources are bf16 with the channel contiguous: packed
+        [T, H, 128], padded [B, S_max, H, 128] (pass ``src_seq_start``), or any
+        strided view (e.g. slices of a fused [T, 3, H, 128] projection).
+        Returns packed uint8 E4M3 codes [T, H, 128]."""
+        for name, t in (("q", q), ("k", k), ("v", v)):
+            _require_cuda(t, name)
+            if t.dtype != torch.bfloat16:
+                raise ValueError(f"{name} must be bfloat16")
+        if q.shape != k.shape or q.shape != v.shape or q.stride() != k.stride() or \
+                q.stride() != v.stride():
+            raise ValueError("q, k, v must share shape and strides")
+        if q.shape[-1] != HEAD_DIM or q.stride(-1) != 1:
+            raise ValueError("head_dim must be 128 and contiguous")
+        H = q.shape[-2]
+        head_stride, tok_stride = q.stride(-2), q.stride(-3)
+        cu = _cu_tensor(cu_seqlens, q.device)
+        B = cu.numel() - 1
+        if total_tokens is None:
+            if src_seq_start is not None:
+                raise ValueError("total_tokens is required with a padded source")
+            total_tokens = q.shape[-3] if q.dim() == 3 else q.shape[0] * q.shape[1]
+        sss = None
+        if src_seq_start is not None:
+            sss = _cu_tensor(src_seq_start, q.device)
+        if out is None:
+            out = [torch.empty((total_tokens, H, HEAD_DIM), dtype=torch.uint8, device=q.device)
+                   for _ in range(3)]
+        _check(lib().fp8attn_quantize_qkv(
+            self._h, layer, mode, _ptr(q), _ptr(k), _ptr(v), tok_stride, head_stride, _ptr(sss),
+            _ptr(cu), B, int(max_seqlen), int(total_tokens), H, HEAD_DIM, _ptr(out[0]),
+            _ptr(out[1]), _ptr(out[2]), ctypes.c_void_p(_stream(stream, q.device))),
+            "fp8attn_quantize_qkv")
+        return out[0], out[1], out[2]
+
+    def amax_ring_update(self, layer: int, amax3: torch.Tensor, stream=None) -> None:
+        """Push three device-side fp32 amax values (q, k, v) into the rings."""
+        _require_cuda(amax3, "amax3")
+        if amax3.dtype != torch.float32 or amax3.numel() != 3:
+            raise ValueError("amax3 must be 3 fp32 values")
+        _check(lib().fp8attn_amax_ring_update(self._h, layer, _ptr(amax3.contiguous()),
+                                              ctypes.c_void_p(_stream(stream, self.device))),
+               "fp8attn_amax_ring_update")
+
+    def set_static_scales(self, layer: int, q: float, k: float, v: float, stream=None) -> None:
+        _check(lib().fp8attn_set_static_scales(self._h, layer, float(q), float(k), float(v),
+                                               ctypes.c_void_p(_stream(stream, self.device))),
+               "fp8attn_set_static_scales")
+
+    def clear_static_scales(self, layer: int) -> None:
+        _check(lib().fp8attn_clear_static_scales(self._h, layer), "fp8attn_clear_static_scales")
+
+    def has_static_scales(self, layer: int) -> bool:
+        r = lib().fp8attn_has_static_scales(self._h, layer)
+        if r < 0:
+            raise FP8AttnError(1, "fp8attn_has_static_scales")
+        return bool(r)
+
+    def export_static_scales(self, margin: float = DEFAULT_MARGIN, stream=None) -> np.ndarray:
+        """[num_layers, 3] float32: fl32(max(ring) * margin) per layer and tensor."""
+        out = np.zeros((self.num_layers, 3), dtype=np.float32)
+        _check(lib().fp8attn_export_static_scales(
+            self._h, float(margin), out.ctypes.data_as(ctypes.c_void_p),
+            ctypes.c_void_p(_stream(stream, self.device))), "fp8attn_export_static_scales")
+        return out
+
+    def descale_ptr(self, layer: int) -> int:
+        p = lib().fp8attn_descale_ptr(self._h, layer)
+        if not p:
+            raise FP8AttnError(1, "fp8attn_descale_ptr")
+        return int(p)
+
+    def quant_scale_ptr(self, layer: int) -> int:
+        p = lib().fp8attn_quant_scale_ptr(self._h, layer)
+        if not p:
+            raise FP8AttnError(1, "fp8attn_quant_scale_ptr")
+        return int(p)
+
+    def get_ring_state(self, layer: int, stream=None) -> Tuple[np.ndarray, np.ndarray]:
+        slots = np.zeros((3, RING_LENGTH), dtype=np.float32)
+        meta = np.zeros((3, 2), dtype=np.uint32)
+        _check(lib().fp8attn_get_ring_state(self._h, layer, slots.ctypes.data_as(ctypes.c_void_p),
+                                            meta.ctypes.data_as(ctypes.c_void_p),
+                                            ctypes.c_void_p(_stream(stream, self.device))),
+               "fp8attn_get_ring_state")
+        return slots, meta
+
+    def set_ring_state(self, layer: int, slots: np.ndarray, meta: np.ndarray, stream=None) -> None:
+        s = np.ascontiguousarray(slots, dtype=np.float32).reshape(3, RING_LENGTH)
+        m = np.ascontiguousarray(meta, dtype=np.uint32).reshape(3, 2)
+        _check(lib().fp8attn_set_ring_state(self._h, layer, s.ctypes.data_as(ctypes.c_void_p),
+                                            m.ctypes.data_as(ctypes.c_void_p),
+                                            ctypes.c_void_p(_stream(stream, self.device))),
+               "fp8attn_set_ring_state")
+
+    def get_scales(self, layer: int, stream=None) -> Tuple[np.ndarray, np.ndarray]:
+        """(qs[3], ds[3]) currently held for the layer."""
+        out = np.zeros(6, dtype=np.float32)
+        _check(lib().fp8attn_get_scales(self._h, layer, out.ctypes.data_as(ctypes.c_void_p),
+                                        ctypes.c_void_p(_stream(stream, self.device))),
+               "fp8attn_get_scales")
+        return out[:3].copy(), out[3:].copy()
+
+    def get_error(self, stream=None) -> int:
+        """Read and clear the device error word; returns the status code."""
+        return int(lib().fp8attn_get_error(self._h, ctypes.c_void_p(_stream(stream, self.device))))
+
+    def select_mode(self, layer: int, skip_mask: Optional[np.ndarray] = None) -> int:
+        m = None
+        if skip_mask is not None:
+            m = np.ascontiguousarray(skip_mask, dtype=np.uint8)
+        r = lib().fp8attn_select_mode(self._h, None if m is None else m.ctypes.data_as(ctypes.c_void_p),
+                                      layer)
+        if r < 0:
+            raise FP8AttnError(1, "fp8attn_select_mode")
+        return r
+
+
+# ---------------------------------------------------------------------------
+# attention
+# ---------------------------------------------------------------------------
+
+def _attn_common(q, k, v, cu_seqlens, out, dtype):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _require_cuda(t, name)
+        if t.dtype != dtype or not t.is_contiguous() or t.dim() != 3 or t.shape[-1] != HEAD_DIM:
+            raise ValueError(f"{name} must be a contiguous [T, H, 128] {dtype} tensor")
+    if q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must have the same shape")
+    T, H, _ = q.shape
+    cu = _cu_tensor(cu_seqlens, q.device)
+    if out is None:
+        out = torch.empty((T, H, HEAD_DIM), dtype=torch.bfloat16, device=q.device)
+    return T, H, cu, out
+
+
+def varlen_fwd(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, cu_seqlens,
+               max_seqlen: int, descale, softmax_scale: float = 0.0,
+               out: Optional[torch.Tensor] = None, error: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    """FP8 attention on packed E4M3 [T, H, 128] codes.  ``descale`` is a device
+    pointer (int, e.g. ``Context.descale_ptr(layer)``) or a 3-element fp32 CUDA
+    tensor {ds_q, ds_k, ds_v}.  Returns bf16 [T, H, 128]."""
+    T, H, cu, out = _attn_common(q8, k8, v8, cu_seqlens, out, torch.uint8)
+    if isinstance(descale, torch.Tensor):
+        _require_cuda(descale, "descale")
+        if descale.dtype != torch.float32 or descale.numel() != 3 or not descale.is_contiguous():
+            raise ValueError("descale must be 3 contiguous fp32 values")
+        dptr = ctypes.c_void_p(descale.data_ptr())
+    else:
+        dptr = ctypes.c_void_p(int(descale))
+    _check(lib().fp8attn_varlen_fwd(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(cu), cu.numel() - 1,
+                                    int(max_seqlen), T, H, HEAD_DIM, dptr, float(softmax_scale),
+                                    _ptr(out), _ptr(error),
+                                    ctypes.c_void_p(_stream(stream, q8.device))),
+           "fp8attn_varlen_fwd")
+    return out
+
+
+def varlen_fwd_bf16(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens,
+                    max_seqlen: int, softmax_scale: float = 0.0,
+                    out: Optional[torch.Tensor] = None, error: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """Native bf16 attention for skipped layers (same kernel, bf16 MMAs)."""
+    T, H, cu, out = _attn_common(q, k, v, cu_seqlens, out, torch.bfloat16)
+    _check(lib().fp8attn_varlen_fwd_bf16(_ptr(q), _ptr(k), _ptr(v), _ptr(cu), cu.numel() - 1,
+                                         int(max_seqlen), T, H, HEAD_DIM, float(softmax_scale),
+                                         _ptr(out), _ptr(error),
+                                         ctypes.c_void_p(_stream(stream, q.device))),
+           "fp8attn_varlen_fwd_bf16")
+    return out
+
+
+def read_error_word(error: torch.Tensor, stream=None) -> int:
+    """Read and clear an attention error word (int32 CUDA tensor)."""
+    _require_cuda(error, "error")
+    return int(lib().fp8attn_read_error_word(_ptr(error),
+                                             ctypes.c_void_p(_stream(stream, error.device))))
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def parse_selector(text: Optional[str], max_index: int) -> set:
+    """Indices selected by "0,1,4-6"-style selectors (via the C parser)."""
+    mask = np.zeros(max(int(max_index), 1), dtype=np.uint8)
+    raw = None if text is None else text.encode()
+    _check(lib().fp8attn_parse_selector(raw, int(max_index), mask.ctypes.data_as(ctypes.c_void_p)),
+           "fp8attn_parse_selector")
+    return set(int(i) for i in np.nonzero(mask[:max_index])[0])
+
+
+def e4m3_encode(x: torch.Tensor, scale: float = 1.0, stream=None) -> torch.Tensor:
+    """E4M3 codes of fl32(x * scale) for an fp32 CUDA tensor (the kernel's cast)."""
+    _require_cuda(x, "x")
+    if x.dtype != torch.float32:
+        raise ValueError("x must be float32")
+    x = x.contiguous()
+    out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    _check(lib().fp8attn_e4m3_encode(_ptr(x), x.numel(), float(scale), _ptr(out),
+                                     ctypes.c_void_p(_stream(stream, x.device))),
+           "fp8attn_e4m3_encode")
+    return out
+
+
+def launch_count() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(lib().fp8attn_launch_count())
+
+
+_ALIASES = {"q": ("q", "q_scale"), "k": ("k", "k_scale"), "v": ("v", "v_scale")}
+
+
+def load_scale_file(path: str) -> Dict[str, Tuple[float, float, float]]:
+    """Read a per-layer {"q","k","v"} scale map (``q_scale``/``k_scale``/
+    ``v_scale`` accepted as aliases), as in the vLLM FP8 ViT page's scale
+    file format section."""
+    with open(path) as f:
+        raw = json.load(f)
+    out = {}
+    for name, entry in raw.items():
+        vals = []
+        for t in ("q", "k", "v"):
+            keys = [k for k in _ALIASES[t] if k in entry]
+            if not keys:
+                raise ValueError(f"layer {name!r} has no {t} value")
+            vals.append(float(entry[keys[0]]))
+        out[name] = tuple(vals)
+    return out
+
+
+def save_scale_file(path: str, layer_names: Sequence[str], values: np.ndarray) -> None:
+    """Write exported values ([L, 3]) as a per-layer {"q","k","v"} map."""
+    values = np.asarray(values, dtype=np.float32).reshape(len(layer_names), 3)
+    data = {n: {"q": float(v[0]), "k": float(v[1]), "v": float(v[2])}
+            for n, v in zip(layer_names, values)}
+    with open(path, "w") as f:
+        json.dump(data, f, indent=2)

@@ -1,0 +1,458 @@
+// Varlen, non-causal flash-attention forward on tcgen05 tensor cores.
+//
+// FP8 (E4M3) instantiation: the quantised Q/K/V feed the attention operator
+// (vLLM-Omni docs, "Quantized KV Cache", overview; vLLM docs, "FP8 ViT
+// encoder attention": per-tensor scales).  BF16 instantiation: the same
+// kernel on native bf16 inputs for skipped layers (vLLM-Omni parameters
+// table: selected layers keep the native dtype).
+//
+// One CTA owns two 128-row query tiles of one (sequence, head) and streams
+// that sequence's 128-key K/V tiles once for both:
+//   warp 8       TMA producer: Q tiles once, then a ring of K/V stages
+//   warp 9       MMA issuer (one lane): S_i = Q_i K^T into TMEM, then
+//                O_i += P_i V from TMEM (P) and shared memory (V, MN-major)
+//   warps 0-3    softmax for query tile 0, warps 4-7 for tile 1: one thread
+//                per query row (= TMEM lane), running max, exp2 with the
+//                descales folded into one FMA, row sum of the unquantised
+//                p, P written back into the S columns, O rescaled in TMEM
+//                when the row max grows, and the bf16 epilogue.
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512);
+// P_i aliases the first 32 (fp8) or 64 (bf16) columns of S_i.  The MMAs of
+// one thread execute in issue order, so S_i(j+1) never overwrites P_i(j)
+// before PV_i(j) has read it, and the arrival of S_i(j+1) also means
+// PV_i(j) has finished (O_i is stable for the rescale).
+//
+// P rule (pages silent; fixed here): p' = 2^(s*c - m + 8) = 256 p with c =
+// ds_q ds_k softmax_scale log2(e) and m the running max of s*c; P = e4m3(p')
+// for the PV product; l accumulates the unquantised p'; out = O ds_v / l.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+#include "state.cuh"
+
+namespace fp8attn {
+
+namespace {
+
+constexpr int kThreadsAttn = 320;
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <bool kFp8>
+struct AttnCfg {
+  static constexpr int kStages = kFp8 ? 4 : 2;
+  static constexpr int kTile = kFp8 ? 16384 : 32768;   // bytes of a 128x128 tile
+  static constexpr int kPCols = kFp8 ? 32 : 64;        // TMEM columns of a P tile
+  static constexpr int kKSteps = kFp8 ? 4 : 8;         // MMAs per 128-deep product
+  static constexpr int kSmemTiles = 2 + 2 * kStages;
+  static constexpr int kSmemBytes = kSmemTiles * kTile + 1024 /*barriers*/ + 1024 /*align*/;
+};
+
+struct AttnParams {
+  const int32_t* cu;
+  int B, H, max_seqlen, n_qblk;   // n_qblk = query blocks of 256 rows per sequence
+  int64_t T;
+  const float* descale;
+  float softmax_scale;
+  __nv_bfloat16* out;
+  int32_t* err;
+};
+
+struct Barriers {
+  uint64_t q_full;
+  uint64_t k_full[4];
+  uint64_t v_full[4];
+  uint64_t kv_empty[4];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_done[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ void note_error(AttnParams& p, Barriers& bars, uint32_t bit) {
+  bars.abort_flag = 1;
+  if (p.err) atomicOr(reinterpret_cast<unsigned int*>(p.err), bit);
+}
+
+template <bool kFp8>
+__global__ void __launch_bounds__(kThreadsAttn, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, AttnParams p) {
+  using C = AttnCfg<kFp8>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sq = smem;                                   // 2 tiles
+  uint8_t* sk = smem + 2 * C::kTile;                    // kStages tiles
+  uint8_t* sv = smem + (2 + C::kStages) * C::kTile;     // kStages tiles
+  Barriers& bars = *reinterpret_cast<Barriers*>(smem + C::kSmemTiles * C::kTile);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work item: (sequence b, head h, query block qb of 256 rows) ----
+  const int qb = blockIdx.x % p.n_qblk;
+  const int bh = blockIdx.x / p.n_qblk;
+  const int h = bh % p.H;
+  const int b = bh / p.H;
+  const int seq0 = __ldg(p.cu + b);
+  const int seq1 = __ldg(p.cu + b + 1);
+  const int len = seq1 - seq0;
+  if (seq0 < 0 || len < 0 || len > p.max_seqlen || static_cast<int64_t>(seq1) > p.T) {
+    if (threadIdx.x == 0 && qb == 0 && p.err)
+      atomicOr(reinterpret_cast<unsigned int*>(p.err), kErrSeqlens);
+    return;
+  }
+  const int q0 = qb * 256;
+  if (q0 >= len) return;
+  const int nkv = (len + 127) / 128;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars.q_full, 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&bars.k_full[s], 1);
+      mbar_init(&bars.v_full[s], 1);
+      mbar_init(&bars.kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.s_full[i], 1);
+      mbar_init(&bars.p_full[i], 128);
+      mbar_init(&bars.o_done[i], 1);
+    }
+    mbar_init(&bars.drain, 1);
+    bars.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&bars.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars.tmem_base;
+  const volatile int* abort_flag = &bars.abort_flag;
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ producer
+    const bool leader = lane == 0;
+    if (leader) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_expect_tx(&bars.q_full, 2 * C::kTile);
+      for (int i = 0; i < 2; ++i) {
+        if (kFp8) {
+          tma_load_3d(sq + i * C::kTile, &tm_q, &bars.q_full, 0, h, seq0 + q0 + 128 * i);
+        } else {
+          tma_load_3d(sq + i * C::kTile, &tm_q, &bars.q_full, 0, h, seq0 + q0 + 128 * i);
+          tma_load_3d(sq + i * C::kTile + 16384, &tm_q, &bars.q_full, 64, h, seq0 + q0 + 128 * i);
+        }
+      }
+    }
+    int issued = 0;
+    for (int j = 0; j < nkv; ++j) {
+      const int st = j % C::kStages;
+      if (j >= C::kStages) {
+        if (!mbar_wait(&bars.kv_empty[st], ((j / C::kStages) - 1) & 1, abort_flag)) {
+          if (leader) note_error(p, bars, kErrTimeout);
+          break;
+        }
+      }
+      if (leader) {
+        const int tok = seq0 + 128 * j;
+        mbar_expect_tx(&bars.k_full[st], C::kTile);
+        tma_load_3d(sk + st * C::kTile, &tm_k, &bars.k_full[st], 0, h, tok);
+        if (!kFp8) tma_load_3d(sk + st * C::kTile + 16384, &tm_k, &bars.k_full[st], 64, h, tok);
+        mbar_expect_tx(&bars.v_full[st], C::kTile);
+        tma_load_3d(sv + st * C::kTile, &tm_v, &bars.v_full[st], 0, h, tok);
+        if (!kFp8) tma_load_3d(sv + st * C::kTile + 16384, &tm_v, &bars.v_full[st], 64, h, tok);
+      }
+      __syncwarp();
+      issued = j + 1;
+    }
+    // make sure no copy is still landing when the CTA leaves
+    for (int j = (issued > C::kStages ? issued - C::kStages : 0); j < issued; ++j) {
+      const int st = j % C::kStages;
+      mbar_wait(&bars.k_full[st], (j / C::kStages) & 1, nullptr);
+      mbar_wait(&bars.v_full[st], (j / C::kStages) & 1, nullptr);
+    }
+    mbar_wait(&bars.q_full, 0, nullptr);
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    const bool leader = lane == 0;
+    const uint32_t id_qk = make_idesc(kFp8 ? 0 : 1, kFp8 ? 0 : 1, 128, 0);
+    const uint32_t id_pv = make_idesc(kFp8 ? 0 : 1, kFp8 ? 0 : 1, 128, 1);
+    const uint32_t tS[2] = {tmem + 0, tmem + 128};
+    const uint32_t tO[2] = {tmem + 256, tmem + 384};
+    const uint32_t q_addr = smem_u32(sq), k_addr = smem_u32(sk), v_addr = smem_u32(sv);
+    auto issue_s = [&](int i, int st) {
+      if (leader) {
+#pragma unroll
+        for (int kk = 0; kk < C::kKSteps; ++kk) {
+          // K-major 128B-swizzled operands: 32 bytes of K per MMA; bf16 tiles
+          // hold two 64-column halves 16 KB apart
+          const uint32_t koff = kFp8 ? 32 * kk : (kk / 4) * 16384 + 32 * (kk % 4);
+          const uint64_t ad = make_sdesc_sw128(q_addr + i * C::kTile + koff, 16, 1024);
+          const uint64_t bd = make_sdesc_sw128(k_addr + st * C::kTile + koff, 16, 1024);
+          if (kFp8) mma_f8_ss(tS[i], ad, bd, id_qk, kk > 0);
+          else mma_bf16_ss(tS[i], ad, bd, id_qk, kk > 0);
+        }
+        mma_commit(&bars.s_full[i]);
+      }
+      __syncwarp();
+    };
+    auto issue_pv = [&](int i, int st, int j) {
+      if (leader) {
+#pragma unroll
+        for (int kk = 0; kk < C::kKSteps; ++kk) {
+          // V is MN-major: K (keys) advances by 32 (fp8) or 16 (bf16) rows of
+          // 128 bytes; the second 64-column half of a bf16 tile sits 16 KB on
+          const uint32_t voff = kFp8 ? 4096 * kk : 2048 * kk;
+          const uint64_t bd = make_sdesc_sw128(v_addr + st * C::kTile + voff, 16384, 1024);
+          if (kFp8) mma_f8_ts(tO[i], tS[i] + 8 * kk, bd, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          else mma_bf16_ts(tO[i], tS[i] + 8 * kk, bd, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+      }
+      __syncwarp();
+    };
+    bool ok = mbar_wait(&bars.q_full, 0, abort_flag) && mbar_wait(&bars.k_full[0], 0, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      issue_s(0, 0);
+      issue_s(1, 0);
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int st = j % C::kStages;
+        const int st1 = (j + 1) % C::kStages;
+        ok = mbar_wait(&bars.v_full[st], (j / C::kStages) & 1, abort_flag) &&
+             mbar_wait(&bars.p_full[0], j & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(0, st, j);
+        if (j + 1 == nkv && leader) mma_commit(&bars.o_done[0]);
+        if (j + 1 < nkv) {
+          ok = mbar_wait(&bars.k_full[st1], ((j + 1) / C::kStages) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(0, st1);
+        }
+        ok = mbar_wait(&bars.p_full[1], j & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(1, st, j);
+        if (leader) {
+          mma_commit(&bars.kv_empty[st]);
+          if (j + 1 == nkv) mma_commit(&bars.o_done[1]);
+        }
+        __syncwarp();
+        if (j + 1 < nkv) issue_s(1, st1);
+      }
+    }
+    if (!ok && leader) note_error(p, bars, kErrTimeout);
+    // drain: every MMA this thread issued has completed before TMEM is freed
+    if (leader) mma_commit(&bars.drain);
+    __syncwarp();
+    mbar_wait(&bars.drain, 0, nullptr);
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int wg = warp >> 2;             // query tile 0 or 1
+    const int wq = warp & 3;              // TMEM lane quadrant
+    const int row = 32 * wq + lane;       // row within the query tile
+    const uint32_t lane_off = static_cast<uint32_t>(32 * wq) << 16;
+    const uint32_t tS = tmem + 128 * wg + lane_off;
+    const uint32_t tO = tmem + 256 + 128 * wg + lane_off;
+    float cscale = p.softmax_scale * kLog2e;
+    float ds_v = 1.0f;
+    if (kFp8) {
+      cscale = __ldg(p.descale + 0) * __ldg(p.descale + 1) * cscale;
+      ds_v = __ldg(p.descale + 2);
+    }
+    const float p_off = kFp8 ? 8.0f : 0.0f;   // 2^8 = 256: P scale for E4M3
+    float m_run = -INFINITY;
+    float l_run = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      if (!mbar_wait(&bars.s_full[wg], j & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t u[128];
+      tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+      tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&u[64]));
+      tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&u[96]));
+      tmem_ld_wait();
+      const int valid = len - 128 * j;
+      if (valid < 128) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= valid) u[c] = 0xFF800000u;   // -inf: key beyond the sequence
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(u[c]));
+      const float m_new = fmaxf(m_run, mx * cscale);
+      const float neg = p_off - m_new;
+      float sum = 0.0f;
+      uint32_t pw[C::kPCols];
+      if (kFp8) {
+#pragma unroll
+        for (int c = 0; c < 128; c += 4) {
+          const float e0 = ex2_approx(fmaf(__uint_as_float(u[c + 0]), cscale, neg));
+          const float e1 = ex2_approx(fmaf(__uint_as_float(u[c + 1]), cscale, neg));
+          const float e2 = ex2_approx(fmaf(__uint_as_float(u[c + 2]), cscale, neg));
+          const float e3 = ex2_approx(fmaf(__uint_as_float(u[c + 3]), cscale, neg));
+          sum += (e0 + e1) + (e2 + e3);
+          pw[c / 4] = static_cast<uint32_t>(cvt_e4m3x2(e0, e1)) |
+                      (static_cast<uint32_t>(cvt_e4m3x2(e2, e3)) << 16);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          const float e0 = ex2_approx(fmaf(__uint_as_float(u[c + 0]), cscale, neg));
+          const float e1 = ex2_approx(fmaf(__uint_as_float(u[c + 1]), cscale, neg));
+          sum += e0 + e1;
+          const __nv_bfloat162 pr = __floats2bfloat162_rn(e0, e1);
+          pw[c / 2] = *reinterpret_cast<const uint32_t*>(&pr);
+        }
+      }
+      const float alpha = ex2_approx(m_run - m_new);   // 0 on the first tile
+      l_run = l_run * alpha + sum;
+      tmem_st32(tS + 0, *reinterpret_cast<const uint32_t(*)[32]>(&pw[0]));
+      if (!kFp8) tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pw[32]));
+      // O_i is stable here (PV_i(j-1) finished before S_i(j) was written)
+      if (j > 0 && __any_sync(0xFFFFFFFFu, m_new > m_run)) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+          tmem_st32(tO + 32 * c, o);
+        }
+      }
+      m_run = m_new;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars.p_full[wg]);
+    }
+    if (!ok) {
+      if (lane == 0) note_error(p, bars, kErrTimeout);
+    } else if (mbar_wait(&bars.o_done[wg], 0, abort_flag)) {
+      // ---- epilogue: out = O * ds_v / l, bf16, valid rows only
+      tc_fence_after();
+      const int qrow = q0 + 128 * wg + row;
+      const bool store = qrow < len;
+      const float inv = ds_v / l_run;
+      __nv_bfloat16* dst =
+          p.out + (static_cast<int64_t>(seq0 + qrow) * p.H + h) * kHeadDim;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * c, o);
+        tmem_ld_wait();
+        uint32_t w[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          const __nv_bfloat162 pr = __floats2bfloat162_rn(__uint_as_float(o[2 * x]) * inv,
+                                                          __uint_as_float(o[2 * x + 1]) * inv);
+          w[x] = *reinterpret_cast<const uint32_t*>(&pr);
+        }
+        if (store) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) d4[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+        }
+      }
+    } else if (lane == 0) {
+      note_error(p, bars, kErrTimeout);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+// [T, H, 128] tensor viewed as (channel, head, token); 128-token boxes of
+// 128 bytes of channels, 128-byte swizzle.
+bool make_qkv_map(CUtensorMap* m, const void* base, int64_t T, int H, bool bf16) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t esz = bf16 ? 2 : 1;
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
+  cuuint64_t strides[2] = {128 * esz, static_cast<cuuint64_t>(H) * 128 * esz};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(bf16 ? 64 : 128), 1, 128};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+            const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool kFp8>
+cudaError_t launch_attention_t(const AttnLaunch& a, int64_t T, cudaStream_t stream) {
+  using C = AttnCfg<kFp8>;
+  CUtensorMap mq, mk, mv;
+  if (!make_qkv_map(&mq, a.q, T, a.heads, !kFp8) || !make_qkv_map(&mk, a.k, T, a.heads, !kFp8) ||
+      !make_qkv_map(&mv, a.v, T, a.heads, !kFp8))
+    return cudaErrorInvalidValue;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<kFp8>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  AttnParams p;
+  p.cu = a.cu;
+  p.B = a.batch;
+  p.H = a.heads;
+  p.max_seqlen = a.max_seqlen;
+  p.n_qblk = (a.max_seqlen + 255) / 256;
+  p.T = T;
+  p.descale = a.descale;
+  p.softmax_scale = a.softmax_scale;
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.err = a.err;
+  const int64_t grid = static_cast<int64_t>(p.n_qblk) * a.heads * a.batch;
+  if (grid <= 0) return cudaSuccess;
+  if (grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
+  attn_fwd_kernel<kFp8><<<static_cast<unsigned>(grid), kThreadsAttn, C::kSmemBytes, stream>>>(
+      mq, mk, mv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const AttnLaunch& a, int64_t total_tokens, cudaStream_t stream) {
+  if (a.bf16) return launch_attention_t<false>(a, total_tokens, stream);
+  return launch_attention_t<true>(a, total_tokens, stream);
+}
+
+}  // namespace fp8attn

@@ -1,0 +1,44 @@
+// Internal launcher interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace fp8attn {
+
+struct QuantLaunch {
+  const void* src[3];            // bf16 q, k, v
+  void* dst[3];                  // E4M3 q8, k8, v8 (packed [T, H, 128])
+  int64_t tok_stride;            // elements
+  int64_t head_stride;           // elements
+  const int32_t* cu;             // device [batch + 1]
+  const int32_t* src_seq_start;  // device [batch] or null
+  int batch, heads, max_seqlen;
+  int64_t total_tokens;          // must equal cu[batch]
+  int dynamic;                   // 1 = ring mode, 0 = static bounds
+  void* gs;                      // GlobalState*
+  void* ls;                      // LayerState*
+};
+
+cudaError_t launch_quantize(const QuantLaunch& q, cudaStream_t stream);
+cudaError_t launch_ring_update(void* ls, void* gs, const float* amax3, cudaStream_t stream);
+cudaError_t launch_rescale_from_ring(void* ls, cudaStream_t stream);
+cudaError_t launch_encode(const float* in, int64_t n, float scale, void* out,
+                          cudaStream_t stream);
+
+struct AttnLaunch {
+  const void* q;                 // E4M3 or bf16 [T, H, 128]
+  const void* k;
+  const void* v;
+  const int32_t* cu;             // device [batch + 1]
+  int batch, heads, max_seqlen;
+  const float* descale;          // device {ds_q, ds_k, ds_v} (fp8 only)
+  float softmax_scale;
+  void* out;                     // bf16 [T, H, 128]
+  int32_t* err;                  // device error word or null
+  int bf16;                      // 1 = native bf16 inputs (skip-layer path)
+};
+
+cudaError_t launch_attention(const AttnLaunch& p, int64_t total_tokens, cudaStream_t stream);
+
+}  // namespace fp8attn

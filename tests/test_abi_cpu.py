@@ -1,0 +1,112 @@
+"""The C-ABI library builds, loads without a GPU and exports every symbol
+that include/fp8attn.h declares; host-only entry points (selector parser,
+status strings, sizes, argument checks) work on the CPU."""
+import ctypes
+import json
+import os
+import re
+
+import numpy as np
+import pytest
+
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "fp8attn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from quantization_amax_reduce_b200 import build
+    build.build()
+    import quantization_amax_reduce_b200 as qar
+    return qar.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(fp8attn_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 20
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_status_strings_and_sizes(L):
+    assert L.fp8attn_status_string(0) == b"ok"
+    assert L.fp8attn_status_string(6) == b"inconsistent cu_seqlens"
+    assert L.fp8attn_ring_length() == 16
+    assert L.fp8attn_workspace_bytes(0) == 0
+    assert L.fp8attn_workspace_bytes(24) == 256 + 24 * 320
+
+
+def test_selector_parser_golden(L, golden_dir):
+    import quantization_amax_reduce_b200 as qar
+    g = json.load(open(os.path.join(golden_dir, "selectors.json")))
+    for c in g["cases"]:
+        assert qar.parse_selector(c["text"], c["max_index"]) == set(c["expect"])
+    for c in g["invalid"]:
+        with pytest.raises(qar.FP8AttnError):
+            qar.parse_selector(c["text"], c["max_index"])
+    assert qar.parse_selector(None, 4) == set()
+    assert qar.parse_selector("  ", 4) == set()
+    assert qar.parse_selector(" 1 , 3 - 4 ", 5) == {1, 3, 4}
+
+
+def test_selector_parser_agrees_with_oracle_on_random_strings(L):
+    import oracle
+    import quantization_amax_reduce_b200 as qar
+    rng = np.random.Generator(np.random.PCG64(3))
+    alphabet = list("0123456789,- ")
+    for _ in range(3000):
+        s = "".join(rng.choice(alphabet, size=rng.integers(0, 9)))
+        try:
+            want = oracle.parse_selector(s, 30)
+        except ValueError:
+            want = None
+        try:
+            got = qar.parse_selector(s, 30)
+        except qar.FP8AttnError:
+            got = None
+        assert got == want, repr(s)
+
+
+def test_host_argument_checks_need_no_gpu(L):
+    P = ctypes.c_void_p
+    # null context / bad layer are rejected before any CUDA call
+    assert L.fp8attn_quantize_qkv(None, 0, 0, P(16), P(16), P(16), 1024, 128, None, P(16), 1,
+                                  8, 8, 8, 128, P(16), P(16), P(16), None) == 1
+    # head_dim other than 128 is unsupported
+    assert L.fp8attn_varlen_fwd(P(16), P(16), P(16), P(16), 1, 8, 8, 8, 64, P(16), 0.0, P(16),
+                                None, None) == 4
+    # total_tokens beyond batch * max_seqlen is invalid
+    assert L.fp8attn_varlen_fwd(P(16), P(16), P(16), P(16), 1, 8, 9, 8, 128, P(16), 0.0, P(16),
+                                None, None) == 1
+    # misaligned pointers are rejected
+    assert L.fp8attn_varlen_fwd(P(17), P(16), P(16), P(16), 1, 8, 8, 8, 128, P(16), 0.0, P(16),
+                                None, None) == 1
+    # zero tokens is a no-op
+    assert L.fp8attn_varlen_fwd(None, None, None, P(16), 1, 8, 0, 8, 128, None, 0.0, None,
+                                None, None) == 0
+    assert L.fp8attn_create(0, P(256), 1 << 20, None, ctypes.byref(P())) == 1
+    assert L.fp8attn_e4m3_encode(None, 5, 1.0, None, None) == 1
+
+
+def test_scale_file_round_trip(tmp_path, golden_dir):
+    import quantization_amax_reduce_b200 as qar
+    g = json.load(open(os.path.join(golden_dir, "static_scale_file.json")))
+    p = tmp_path / "scales.json"
+    p.write_text(json.dumps(g["map"]))
+    m = qar.load_scale_file(str(p))
+    assert m["visual.blocks.0.attn.attn"] == (224.0, 198.0, 210.0)
+    assert m["visual.blocks.1.attn.attn"] == (218.0, 195.0, 207.0)
+    p2 = tmp_path / "alias.json"
+    p2.write_text(json.dumps(g["alias_map"]))
+    assert qar.load_scale_file(str(p2))["visual.blocks.0.attn.attn"] == (224.0, 198.0, 210.0)
+    out = tmp_path / "saved.json"
+    qar.save_scale_file(str(out), ["a", "b"], np.array([[1.5, 3.0, 4.5], [6.0, 7.5, 9.0]]))
+    assert qar.load_scale_file(str(out)) == {"a": (1.5, 3.0, 4.5), "b": (6.0, 7.5, 9.0)}

@@ -1,0 +1,147 @@
+"""GPU parity of the tcgen05 varlen attention kernels against the oracle.
+
+FP8: vLLM-Omni docs, "Quantized KV Cache", overview (quantised Q/K/V feed a
+full, non-causal attention operator) and vLLM docs, "FP8 ViT encoder
+attention" (per-tensor scales).  BF16: vLLM-Omni parameters table (skipped
+layers keep the native dtype).  Tolerance: max |err| <= 1e-2 and mean |err|
+<= 1e-3 against the oracle's fp64 attention with the same P rule."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+import quantization_amax_reduce_b200 as qar
+from tests.parity import (OracleLayer, assert_attention_close, attention_errors, bits,
+                          sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _codes(T, H, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(T, H, 128, generator=g) * scale
+    return x.to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+CASES = [
+    ([1], 1), ([5], 2), ([128], 1), ([129], 1), ([256], 2), ([257], 1), ([383], 3),
+    ([1000, 17], 2), ([5, 300, 129], 3), ([64, 0, 200, 0], 2), ([513, 1, 255], 1),
+]
+
+
+@pytest.mark.parametrize("lens,H", CASES)
+def test_fp8_attention_small_shapes(lens, H):
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(cu[-1])
+    q8, k8, v8 = (_codes(T, H, s, 6.0) for s in (1, 2, 3))
+    # v ~ N(0, 0.1^2): outputs of the size the workloads produce, so the
+    # absolute tolerance measures the kernel rather than bf16 output rounding
+    ds = torch.tensor([0.05, 0.04, 1.0 / 60.0], dtype=torch.float32)
+    out = qar.varlen_fwd(q8.to(DEV), k8.to(DEV), v8.to(DEV), torch.as_tensor(cu, device=DEV),
+                         max(lens), ds.to(DEV))
+    want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds.tolist())
+    assert_attention_close(out, want, what=f"fp8 {lens} H={H}")
+
+
+@pytest.mark.parametrize("lens,H", CASES[:8])
+def test_bf16_attention_small_shapes(lens, H):
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    q, k, v, _ = synthetic.small_qkv(31, lens, H=H, scale=1.5)
+    v = (v.float() * (1.0 / 15.0)).to(torch.bfloat16)   # v ~ N(0, 0.1^2)
+    out = qar.varlen_fwd_bf16(q.to(DEV), k.to(DEV), v.to(DEV), torch.as_tensor(cu, device=DEV),
+                              max(lens))
+    want = oracle.attention_bf16(bits(q), bits(k), bits(v), cu)
+    assert_attention_close(out, want, what=f"bf16 {lens} H={H}")
+
+
+def test_sharp_softmax_rescales():
+    """Large score range so the running max moves across key tiles (O
+    rescaling in TMEM) and many p fall in E4M3's subnormal range."""
+    lens = [900]
+    H = 2
+    cu = np.array([0, 900], dtype=np.int32)
+    g = torch.Generator().manual_seed(9)
+    # increasing key norms along the sequence: later tiles hold larger maxima
+    ramp = torch.linspace(0.2, 3.0, 900).view(900, 1, 1)
+    q8 = (torch.randn(900, H, 128, generator=g) * 4).to(torch.float8_e4m3fn).view(torch.uint8)
+    k8 = (torch.randn(900, H, 128, generator=g) * 4 * ramp).to(torch.float8_e4m3fn).view(torch.uint8)
+    v8 = (torch.randn(900, H, 128, generator=g) * 4).to(torch.float8_e4m3fn).view(torch.uint8)
+    ds = [0.25, 0.25, 0.025]
+    out = qar.varlen_fwd(q8.to(DEV), k8.to(DEV), v8.to(DEV), torch.as_tensor(cu, device=DEV),
+                         900, torch.tensor(ds, device=DEV))
+    want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds)
+    assert_attention_close(out, want, what="sharp")
+
+
+def test_explicit_softmax_scale():
+    cu = np.array([0, 300], dtype=np.int32)
+    q8, k8, v8 = (_codes(300, 2, s, 3.0) for s in (4, 5, 6))
+    ds = [0.1, 0.1, 0.05]
+    out = qar.varlen_fwd(q8.to(DEV), k8.to(DEV), v8.to(DEV), torch.as_tensor(cu, device=DEV),
+                         300, torch.tensor(ds, device=DEV), softmax_scale=0.3)
+    want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds, scale=0.3)
+    assert_attention_close(out, want, what="scale 0.3")
+
+
+def test_c1_end_to_end_through_the_boundary():
+    q, k, v, cu = synthetic.qkv(1)
+    ctx = qar.Context(1)
+    cu_d = torch.as_tensor(cu, device=DEV)
+    q8, k8, v8 = ctx.quantize_qkv(0, qar.DYNAMIC, q.to(DEV), k.to(DEV), v.to(DEV), cu_d, 256)
+    out = qar.varlen_fwd(q8, k8, v8, cu_d, 256, ctx.descale_ptr(0))
+    ol = OracleLayer()
+    codes = ol.dynamic_pass([bits(q), bits(k), bits(v)], cu, 2)
+    want = oracle.attention_fp8(*codes, cu, [float(x) for x in ol.ds])
+    mx, mean = assert_attention_close(out, want, what="c1")
+    # error against unquantised fp64 attention on the bf16 inputs (reported)
+    ref = oracle.attention_bf16(bits(q), bits(k), bits(v), cu)
+    print("c1 vs oracle max/mean", mx, mean, "vs unquantised", attention_errors(out, ref))
+
+
+def test_c3_full_size_sampled_rows():
+    """The benchmarked configuration: S=8192, 16 heads, static 224/198/210."""
+    q, k, v, cu = synthetic.qkv(3, device=DEV)
+    ctx = qar.Context(1)
+    ctx.set_static_scales(0, 224.0, 198.0, 210.0)
+    cu_d = torch.as_tensor(cu, device=DEV)
+    q8, k8, v8 = ctx.quantize_qkv(0, qar.STATIC, q, k, v, cu_d, 8192)
+    out = qar.varlen_fwd(q8, k8, v8, cu_d, 8192, ctx.descale_ptr(0))
+    rows = sample_rows(cu, 96, seed=3)
+    ds = [float(x) for x in ctx.get_scales(0)[1]]
+    want = oracle.attention_fp8(q8.cpu().numpy(), k8.cpu().numpy(), v8.cpu().numpy(), cu, ds,
+                                rows=rows)
+    assert_attention_close(out, want, rows=rows, what="c3")
+
+
+def test_c2_varlen_after_sixteen_passes_sampled_rows():
+    w = synthetic.WORKLOADS[2]
+    ctx = qar.Context(1)
+    cu = w.cu_seqlens(0)
+    cu_d = torch.as_tensor(cu, device=DEV)
+    max_len = int(np.diff(cu).max())
+    for p in range(w.passes):
+        q, k, v, _ = synthetic.qkv(2, 0, p, device=DEV)
+        q8, k8, v8 = ctx.quantize_qkv(0, qar.DYNAMIC, q, k, v, cu_d, max_len)
+    out = qar.varlen_fwd(q8, k8, v8, cu_d, max_len, ctx.descale_ptr(0))
+    rows = sample_rows(cu, 64, seed=2)
+    ds = [float(x) for x in ctx.get_scales(0)[1]]
+    want = oracle.attention_fp8(q8.cpu().numpy(), k8.cpu().numpy(), v8.cpu().numpy(), cu, ds,
+                                rows=rows)
+    assert_attention_close(out, want, rows=rows, what="c2")
+
+
+def test_bad_cu_seqlens_sets_error_word():
+    cu = torch.tensor([0, 100, 50], dtype=torch.int32, device=DEV)   # decreasing
+    q8 = torch.zeros(300, 1, 128, dtype=torch.uint8, device=DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out = torch.full((300, 1, 128), 7.0, dtype=torch.bfloat16, device=DEV)
+    qar.varlen_fwd(q8, q8, q8, cu, 300, torch.ones(3, device=DEV), out=out, error=err)
+    assert qar.read_error_word(err) == 6
+    assert (out[100:] == 7.0).all()       # the broken sequence wrote nothing
+    assert (out[:100] == 0.0).all()       # the valid one attends to zeros
+    assert qar.read_error_word(err) == 0

@@ -152,3 +152,43 @@ def test_row_subset_equals_full_rows():
     rows = [0, 19, 20, 32, 5]
     sub = oracle.attention_fp8(q8, k8, v8, cu, (0.1, 0.2, 0.3), rows=rows)
     np.testing.assert_array_equal(sub, full[rows])
+
+
+def test_pquant_rule_uses_running_block_max():
+    # 129 keys: keys 0..127 score 0 (block 0), key 128 scores 1 (block 1).
+    # Block 0 is quantised against its own max 0: p = 1 -> 256 is exact, then
+    # carried to the final max 1 by the exact factor e^-1, so p~ = e^-1.
+    # (Against the final max it would be e4m3(256 e^-1) = e4m3(94.18) = 96,
+    # p~ = 0.375.)  Key 128: p~ = 1.  l = 128 e^-1 + 1 (unquantised).
+    D, n = 128, 129
+    q8 = np.zeros((n, 1, D), np.uint8)
+    k8 = np.zeros((n, 1, D), np.uint8)
+    v8 = np.zeros((n, 1, D), np.uint8)
+    q8[:, 0, 0] = 0x38                # q = e_0
+    k8[128, 0, 0] = 0x38              # s_128 = 1
+    v8[128, 0, 1] = 0x38              # v_128 = e_1
+    v8[0, 0, 2] = 0x38                # v_0 = e_2
+    cu = np.array([0, n], dtype=np.int32)
+    o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True,
+                             rows=[5])
+    l = 128 * math.exp(-1.0) + 1.0
+    assert abs(o[0, 0, 1] - 1.0 / l) < 1e-15
+    assert abs(o[0, 0, 2] - math.exp(-1.0) / l) < 1e-15
+    assert abs(o[0, 0, 2] - 0.375 / l) > 1e-4       # not the final-max rule
+
+
+def test_pquant_block_rule_second_block_lower_max():
+    # block 1's scores are all below block 0's max: its running max is the
+    # same as block 0's, so p~ = e4m3(256 e^s)/256 for s = -0.125 there: 224/256
+    D, n = 128, 130
+    q8 = np.zeros((n, 1, D), np.uint8)
+    k8 = np.zeros((n, 1, D), np.uint8)
+    v8 = np.zeros((n, 1, D), np.uint8)
+    q8[:, 0, 0] = 0x38
+    k8[128:, 0, 0] = 0xA0             # s = -0.125 for keys 128, 129
+    v8[129, 0, 3] = 0x38
+    cu = np.array([0, n], dtype=np.int32)
+    o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True,
+                             rows=[0])
+    l = 128 + 2 * math.exp(-0.125)
+    assert abs(o[0, 0, 3] - 0.875 / l) < 1e-15
