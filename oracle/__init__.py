@@ -75,7 +75,7 @@ def lib() -> ctypes.CDLL:
     L.or_export_value.argtypes = [ctypes.POINTER(_Ring), f32]
     L.or_attention_fp8.restype = i32
     L.or_attention_fp8.argtypes = [P, P, P, P, i32, i32, i32, f64, f64, f64, f64,
-                                   i32, i32, P, i64, P, i32]
+                                   i32, i32, P, i64, P, P, i32]
     L.or_attention_bf16.restype = i32
     L.or_attention_bf16.argtypes = [P, P, P, P, i32, i32, i32, f64, P, i64, P, i32]
     _lib = L
@@ -225,13 +225,17 @@ def _rows_arg(rows):
 
 def attention_fp8(q8, k8, v8, cu, ds_qkv: Sequence[float], scale: Optional[float] = None,
                   pquant: bool = True, l_of_quantized: bool = False, rows=None,
-                  nthreads: int = 0) -> np.ndarray:
+                  nthreads: int = 0, return_ambiguity: bool = False):
     """fp64 attention on E4M3 codes [T, H, D]; returns [len(rows) or T, H, D].
 
     With ``pquant`` the PV product uses P quantised per block of 128 keys (in
     sequence order) as e4m3(256 exp(s - m))/256, m the running row max over
     the keys seen so far, carried exactly to the final max M; l is the sum of
-    the unquantised exp(s - M) unless ``l_of_quantized``."""
+    the unquantised exp(s - M) unless ``l_of_quantized``.
+
+    With ``return_ambiguity`` also returns, per output, the largest change
+    that P codes lying within an fp32 evaluation's error of a rounding tie
+    can make (either neighbouring code is a correct result there)."""
     q8 = np.ascontiguousarray(q8, dtype=np.uint8)
     k8 = np.ascontiguousarray(k8, dtype=np.uint8)
     v8 = np.ascontiguousarray(v8, dtype=np.uint8)
@@ -242,11 +246,12 @@ def attention_fp8(q8, k8, v8, cu, ds_qkv: Sequence[float], scale: Optional[float
     r, nr = _rows_arg(rows)
     n = nr if r is not None else int(cu[-1])
     out = np.empty((n, H, D), dtype=np.float64)
+    amb = np.empty((n, H, D), dtype=np.float64) if return_ambiguity else None
     lib().or_attention_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(cu), cu.size - 1, H, D,
                            float(ds_qkv[0]), float(ds_qkv[1]), float(ds_qkv[2]),
                            float(scale), int(bool(pquant)), int(bool(l_of_quantized)),
-                           _ptr(r), nr, _ptr(out), nthreads)
-    return out
+                           _ptr(r), nr, _ptr(out), _ptr(amb), nthreads)
+    return (out, amb) if return_ambiguity else out
 
 
 def attention_bf16(q_u16, k_u16, v_u16, cu, scale: Optional[float] = None, rows=None,

@@ -332,6 +332,7 @@ typedef struct {
     const int64_t* rows;      /* token indices to evaluate (or NULL: all) */
     int64_t nrows;
     double* out;              /* [nrows][H][D] */
+    double* amb;              /* [nrows][H][D] ambiguity allowance, or NULL */
     int64_t next;             /* work counter (rows*H items) */
     pthread_mutex_t lock;
 } att_job;
@@ -349,12 +350,30 @@ static double elem(const att_job* j, const void* base, int64_t t, int h, int d) 
  * factor exp(m_t - M).  l is the sum of the unquantised p = exp(s - M). */
 #define OR_P_BLOCK 128
 
+/* Codes within reach of a rounding tie.  An implementation evaluates
+ * y = 256 exp(s - m) in fp32 (exp2 of s*log2(e) - m*log2(e) + 8), so its y
+ * carries a relative error of a few fp32 roundings of the exponent's terms
+ * plus the exp2 approximation; bound it by
+ *     eps(y) = 2^-20 * (2 + |s| log2(e) + |m| log2(e))
+ * (16x the fp32 rounding of each term).  When [y(1-eps), y(1+eps)] holds a
+ * tie between two E4M3 values, either code is a correct result of the rule;
+ * the caller receives the largest output change such a flip can make. */
+static double code_ambiguity(double y, double s, double m) {
+    const double log2e = 1.4426950408889634;
+    double eps = ldexp(1.0, -20) * (2.0 + fabs(s) * log2e + fabs(m) * log2e);
+    uint8_t lo = or_e4m3_encode(y * (1.0 - eps));
+    uint8_t hi = or_e4m3_encode(y * (1.0 + eps));
+    if (lo == hi) return 0.0;
+    return fabs(or_e4m3_value(hi) - or_e4m3_value(lo)) / 256.0;
+}
+
 static void attend_one(const att_job* j, int64_t ri, int h, double* s_buf) {
     int64_t t = j->rows ? j->rows[ri] : ri;
     int b, d;
     int64_t k0, k1, kk;
     double M = -INFINITY, l = 0.0, m_blk = -INFINITY;
     double* o = j->out + (ri * j->H + h) * (int64_t)j->D;
+    double* a = j->amb ? j->amb + (ri * j->H + h) * (int64_t)j->D : NULL;
     double dsq = j->kind == 0 ? j->ds_q : 1.0;
     double dsk = j->kind == 0 ? j->ds_k : 1.0;
     double dsv = j->kind == 0 ? j->ds_v : 1.0;
@@ -370,6 +389,8 @@ static void attend_one(const att_job* j, int64_t ri, int h, double* s_buf) {
         if (s_buf[kk - k0] > M) M = s_buf[kk - k0];
     }
     for (d = 0; d < j->D; ++d) o[d] = 0.0;
+    if (a)
+        for (d = 0; d < j->D; ++d) a[d] = 0.0;
     for (kk = k0; kk < k1; ++kk) {
         double s = s_buf[kk - k0];
         double p = exp(s - M);
@@ -380,13 +401,21 @@ static void attend_one(const att_job* j, int64_t ri, int h, double* s_buf) {
             for (x = kk; x < e; ++x)
                 if (s_buf[x - k0] > m_blk) m_blk = s_buf[x - k0];
         }
-        if (j->pquant)
-            pt = or_e4m3_value(or_e4m3_encode(256.0 * exp(s - m_blk))) / 256.0 *
-                 exp(m_blk - M);
+        if (j->pquant) {
+            double y = 256.0 * exp(s - m_blk);
+            pt = or_e4m3_value(or_e4m3_encode(y)) / 256.0 * exp(m_blk - M);
+            if (a) {
+                double amb = code_ambiguity(y, s, m_blk) * exp(m_blk - M);
+                if (amb > 0.0)
+                    for (d = 0; d < j->D; ++d) a[d] += amb * fabs(elem(j, j->v, kk, h, d));
+            }
+        }
         l += j->lrule ? pt : p;
         for (d = 0; d < j->D; ++d) o[d] += pt * elem(j, j->v, kk, h, d);
     }
     for (d = 0; d < j->D; ++d) o[d] = o[d] * dsv / l;
+    if (a)
+        for (d = 0; d < j->D; ++d) a[d] = a[d] * dsv / l;
 }
 
 static void* att_worker(void* arg) {
@@ -433,7 +462,7 @@ int or_attention_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
                      const int32_t* cu, int B, int H, int D,
                      double ds_q, double ds_k, double ds_v, double scale,
                      int pquant, int lrule, const int64_t* rows, int64_t nrows,
-                     double* out, int nthreads) {
+                     double* out, double* amb, int nthreads) {
     att_job j;
     memset(&j, 0, sizeof(j));
     j.kind = 0;
@@ -441,7 +470,7 @@ int or_attention_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
     j.cu = cu; j.B = B; j.H = H; j.D = D;
     j.ds_q = ds_q; j.ds_k = ds_k; j.ds_v = ds_v; j.scale = scale;
     j.pquant = pquant; j.lrule = lrule;
-    j.rows = rows; j.nrows = nrows; j.out = out;
+    j.rows = rows; j.nrows = nrows; j.out = out; j.amb = amb;
     return run_attention(&j, nthreads);
 }
 

@@ -44,7 +44,7 @@ def test_fp8_attention_small_shapes(lens, H):
     ds = torch.tensor([0.05, 0.04, 1.0 / 60.0], dtype=torch.float32)
     out = qar.varlen_fwd(q8.to(DEV), k8.to(DEV), v8.to(DEV), torch.as_tensor(cu, device=DEV),
                          max(lens), ds.to(DEV))
-    want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds.tolist())
+    want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds.tolist(), return_ambiguity=True)
     assert_attention_close(out, want, what=f"fp8 {lens} H={H}")
 
 
@@ -74,7 +74,7 @@ def test_sharp_softmax_rescales():
     ds = [0.25, 0.25, 0.025]
     out = qar.varlen_fwd(q8.to(DEV), k8.to(DEV), v8.to(DEV), torch.as_tensor(cu, device=DEV),
                          900, torch.tensor(ds, device=DEV))
-    want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds)
+    want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds, return_ambiguity=True)
     assert_attention_close(out, want, what="sharp")
 
 
@@ -84,7 +84,7 @@ def test_explicit_softmax_scale():
     ds = [0.1, 0.1, 0.05]
     out = qar.varlen_fwd(q8.to(DEV), k8.to(DEV), v8.to(DEV), torch.as_tensor(cu, device=DEV),
                          300, torch.tensor(ds, device=DEV), softmax_scale=0.3)
-    want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds, scale=0.3)
+    want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds, scale=0.3, return_ambiguity=True)
     assert_attention_close(out, want, what="scale 0.3")
 
 
@@ -96,7 +96,7 @@ def test_c1_end_to_end_through_the_boundary():
     out = qar.varlen_fwd(q8, k8, v8, cu_d, 256, ctx.descale_ptr(0))
     ol = OracleLayer()
     codes = ol.dynamic_pass([bits(q), bits(k), bits(v)], cu, 2)
-    want = oracle.attention_fp8(*codes, cu, [float(x) for x in ol.ds])
+    want = oracle.attention_fp8(*codes, cu, [float(x) for x in ol.ds], return_ambiguity=True)
     mx, mean = assert_attention_close(out, want, what="c1")
     # error against unquantised fp64 attention on the bf16 inputs (reported)
     ref = oracle.attention_bf16(bits(q), bits(k), bits(v), cu)
@@ -114,7 +114,7 @@ def test_c3_full_size_sampled_rows():
     rows = sample_rows(cu, 96, seed=3)
     ds = [float(x) for x in ctx.get_scales(0)[1]]
     want = oracle.attention_fp8(q8.cpu().numpy(), k8.cpu().numpy(), v8.cpu().numpy(), cu, ds,
-                                rows=rows)
+                                rows=rows, return_ambiguity=True)
     assert_attention_close(out, want, rows=rows, what="c3")
 
 
@@ -131,7 +131,7 @@ def test_c2_varlen_after_sixteen_passes_sampled_rows():
     rows = sample_rows(cu, 64, seed=2)
     ds = [float(x) for x in ctx.get_scales(0)[1]]
     want = oracle.attention_fp8(q8.cpu().numpy(), k8.cpu().numpy(), v8.cpu().numpy(), cu, ds,
-                                rows=rows)
+                                rows=rows, return_ambiguity=True)
     assert_attention_close(out, want, rows=rows, what="c2")
 
 

@@ -33,7 +33,7 @@ def test_c4_dit_dynamic_full_size():
         assert_codes_equal(g, w, n)
     assert_scales_equal(ctx, 0, ol)
     rows = sample_rows(cu, 24, seed=4)
-    want = oracle.attention_fp8(*codes, cu, [float(x) for x in ol.ds], rows=rows)
+    want = oracle.attention_fp8(*codes, cu, [float(x) for x in ol.ds], rows=rows, return_ambiguity=True)
     assert_attention_close(out, want, rows=rows, what="c4")
     assert ctx.get_error() == 0
 
@@ -105,5 +105,5 @@ def test_c5_calibrate_then_serve():
             assert_codes_equal(g, ww, f"serve layer {l} {n}")
         assert_scales_equal(ctx, l, ols[l])
         out = qar.varlen_fwd(q8, k8, v8, cu_d, max_len, ctx.descale_ptr(l))
-        want = oracle.attention_fp8(*codes, cu, [float(x) for x in ols[l].ds], rows=rows)
+        want = oracle.attention_fp8(*codes, cu, [float(x) for x in ols[l].ds], rows=rows, return_ambiguity=True)
         assert_attention_close(out, want, rows=rows, what=f"serve fp8 layer {l}")

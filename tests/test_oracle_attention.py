@@ -192,3 +192,21 @@ def test_pquant_block_rule_second_block_lower_max():
                              rows=[0])
     l = 128 + 2 * math.exp(-0.125)
     assert abs(o[0, 0, 3] - 0.875 / l) < 1e-15
+
+
+def test_ambiguity_reported_only_at_rounding_ties():
+    # s1 = ln(232/256): y1 = 256 e^{s1} = 232 is the tie between the E4M3
+    # values 224 and 240, so both codes are correct results of the rule and
+    # the oracle reports the one-step change (16/256) * |v1| / l.
+    q8, k8, v8, cu = _two_key_case(0x38)          # k1 = 1.0 * e_0
+    ds_k = math.log(232.0 / 256.0)
+    o, amb = oracle.attention_fp8(q8, k8, v8, cu, (1.0, ds_k, 1.0), scale=1.0, pquant=True,
+                                  return_ambiguity=True)
+    l = 1.0 + 232.0 / 256.0
+    assert abs(amb[0, 0, 1] - (16.0 / 256.0) / l) < 1e-12
+    assert amb[0, 0, 0] == 0.0                    # v1 has no component there
+    # y1 = 225.92 (s1 = -0.125) is far from any tie: no allowance
+    q8, k8, v8, cu = _two_key_case(0xA0)
+    o, amb = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True,
+                                  return_ambiguity=True)
+    assert (amb == 0.0).all()
