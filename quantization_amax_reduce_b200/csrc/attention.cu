@@ -292,33 +292,54 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int c = 0; c < 128; ++c)
           if (c >= valid) u[c] = 0xFF800000u;   // -inf: key beyond the sequence
       }
-      float mx = -INFINITY;
+      // row max: four independent chains of 3-input max
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(u[c]));
+      for (int c = 0; c < 128; c += 8) {
+        mx0 = fmax3(mx0, __uint_as_float(u[c + 0]), __uint_as_float(u[c + 1]));
+        mx1 = fmax3(mx1, __uint_as_float(u[c + 2]), __uint_as_float(u[c + 3]));
+        mx2 = fmax3(mx2, __uint_as_float(u[c + 4]), __uint_as_float(u[c + 5]));
+        mx3 = fmax3(mx3, __uint_as_float(u[c + 6]), __uint_as_float(u[c + 7]));
+      }
+      const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3));
       const float m_new = fmaxf(m_run, mx * cscale);
       const float neg = p_off - m_new;
-      float sum = 0.0f;
+      const uint64_t c2 = f2_pack(cscale, cscale);
+      const uint64_t n2 = f2_pack(neg, neg);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
       uint32_t pw[C::kPCols];
-      if (kFp8) {
 #pragma unroll
-        for (int c = 0; c < 128; c += 4) {
-          const float e0 = ex2_approx(fmaf(__uint_as_float(u[c + 0]), cscale, neg));
-          const float e1 = ex2_approx(fmaf(__uint_as_float(u[c + 1]), cscale, neg));
-          const float e2 = ex2_approx(fmaf(__uint_as_float(u[c + 2]), cscale, neg));
-          const float e3 = ex2_approx(fmaf(__uint_as_float(u[c + 3]), cscale, neg));
-          sum += (e0 + e1) + (e2 + e3);
-          pw[c / 4] = static_cast<uint32_t>(cvt_e4m3x2(e0, e1)) |
-                      (static_cast<uint32_t>(cvt_e4m3x2(e2, e3)) << 16);
+      for (int k = 0; k < 64; ++k) {
+        // exponent argument for columns 2k, 2k+1 in one packed FMA
+        const uint64_t t = f2_fma(f2_pack(__uint_as_float(u[2 * k]), __uint_as_float(u[2 * k + 1])),
+                                  c2, n2);
+        float t0, t1;
+        f2_unpack(t, t0, t1);
+        uint64_t e;
+        if ((k & 7) >= 5) {
+          // 3 of every 8 pairs on the FMA pipe, the rest on the MUFU
+          e = f2_exp2_poly(f2_pack(fmaxf(t0, -126.0f), fmaxf(t1, -126.0f)));
+        } else {
+          e = f2_pack(ex2_approx(t0), ex2_approx(t1));
         }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          const float e0 = ex2_approx(fmaf(__uint_as_float(u[c + 0]), cscale, neg));
-          const float e1 = ex2_approx(fmaf(__uint_as_float(u[c + 1]), cscale, neg));
-          sum += e0 + e1;
-          const __nv_bfloat162 pr = __floats2bfloat162_rn(e0, e1);
-          pw[c / 2] = *reinterpret_cast<const uint32_t*>(&pr);
+        acc[k & 3] = f2_add(acc[k & 3], e);
+        float e0, e1;
+        f2_unpack(e, e0, e1);
+        if (kFp8) {
+          const uint32_t h = cvt_e4m3x2(e0, e1);
+          if (k & 1) pw[k >> 1] |= h << 16;
+          else pw[k >> 1] = h;
+        } else {
+          pw[k] = cvt_bf16x2(e0, e1);
         }
+      }
+      float sum;
+      {
+        float a0, a1, b0, b1;
+        f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
+        (void)b0;
+        (void)b1;
+        sum = a0 + a1;
       }
       const float alpha = ex2_approx(m_run - m_new);   // 0 on the first tile
       l_run = l_run * alpha + sum;
@@ -331,8 +352,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           uint32_t o[32];
           tmem_ld32(tO + 32 * c, o);
           tmem_ld_wait();
+          const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-          for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+          for (int x = 0; x < 32; x += 2) {
+            float o0, o1;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(o[x]), __uint_as_float(o[x + 1])), a2), o0, o1);
+            o[x] = __float_as_uint(o0);
+            o[x + 1] = __float_as_uint(o1);
+          }
           tmem_st32(tO + 32 * c, o);
         }
       }
@@ -357,11 +384,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_ld32(tO + 32 * c, o);
         tmem_ld_wait();
         uint32_t w[16];
+        const uint64_t inv2 = f2_pack(inv, inv);
 #pragma unroll
         for (int x = 0; x < 16; ++x) {
-          const __nv_bfloat162 pr = __floats2bfloat162_rn(__uint_as_float(o[2 * x]) * inv,
-                                                          __uint_as_float(o[2 * x + 1]) * inv);
-          w[x] = *reinterpret_cast<const uint32_t*>(&pr);
+          float o0, o1;
+          f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * x]), __uint_as_float(o[2 * x + 1])), inv2),
+                    o0, o1);
+          w[x] = cvt_bf16x2(o0, o1);
         }
         if (store) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);

@@ -311,4 +311,78 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Two bf16 (round to nearest even), `lo` in the low half.
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// Packed fp32 pairs (sm_100 f32x2 arithmetic) and 3-input max
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair of arguments on the FMA pipe, for arguments in [-126, 8]
+// (callers clamp from below).  Cody-Waite style reduction x = j + f with j
+// = nearest integer (1.5 * 2^23 added and removed), f in [-1/2, 1/2]; 2^f
+// from a degree-5 polynomial fitted here by the Remez exchange algorithm
+// for minimum relative error (2.1e-7 evaluated in fp32); the integer j
+// goes straight into the exponent bits.
+__device__ __forceinline__ uint64_t f2_exp2_poly(uint64_t x) {
+  const uint64_t kShift = f2_pack(12582912.0f, 12582912.0f);        // 1.5 * 2^23
+  const uint64_t kNegShift = f2_pack(-12582912.0f, -12582912.0f);
+  const uint64_t kMinusOne = f2_pack(-1.0f, -1.0f);
+  const uint64_t r = f2_add(x, kShift);                 // j in the low mantissa bits
+  const uint64_t j = f2_add(r, kNegShift);              // j as a float (exact)
+  const uint64_t f = f2_fma(j, kMinusOne, x);           // x - j, exact
+  uint64_t p = f2_pack(1.3276472e-3f, 1.3276472e-3f);
+  p = f2_fma(p, f, f2_pack(9.6755410e-3f, 9.6755410e-3f));
+  p = f2_fma(p, f, f2_pack(5.5507131e-2f, 5.5507131e-2f));
+  p = f2_fma(p, f, f2_pack(2.4022120e-1f, 2.4022120e-1f));
+  p = f2_fma(p, f, f2_pack(6.9314694e-1f, 6.9314694e-1f));
+  p = f2_fma(p, f, f2_pack(1.0000001f, 1.0000001f));
+  uint32_t plo, phi, rlo, rhi;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(plo), "=r"(phi) : "l"(p));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(rlo), "=r"(rhi) : "l"(r));
+  plo += rlo << 23;
+  phi += rhi << 23;
+  uint64_t out;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(out) : "r"(plo), "r"(phi));
+  return out;
+}
+
 }  // namespace fp8attn
