@@ -8,7 +8,7 @@
 #include <new>
 #include <vector>
 
-#include "../../include/fp8attn.h"
+#include "fp8attn.h"
 #include "kernels.h"
 #include "state.cuh"
 

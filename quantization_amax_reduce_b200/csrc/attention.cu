@@ -38,6 +38,14 @@ namespace fp8attn {
 namespace {
 
 constexpr int kThreadsAttn = 320;
+// Softmax scheduling: the two query tiles' softmax warpgroups take turns
+// (tile 0 of key block j, tile 1 of block j, tile 0 of block j+1, ...), so
+// each runs with the SM's exp and FMA pipes to itself while the tensor core
+// works on the other tile's MMAs.
+constexpr bool kAlternate = false;
+// Pairs of columns (of every 8) whose exp2 runs on the FMA pipe (polynomial)
+// instead of the MUFU.
+constexpr int kPolyPairsPer8 = 2;
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -70,6 +78,7 @@ struct Barriers {
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_done[2];
+  uint64_t tok[2];        // softmax turn tokens (tile 1 -> tile 0, tile 0 -> tile 1)
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -124,6 +133,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_init(&bars.s_full[i], 1);
       mbar_init(&bars.p_full[i], 128);
       mbar_init(&bars.o_done[i], 1);
+      mbar_init(&bars.tok[i], 128);
     }
     mbar_init(&bars.drain, 1);
     bars.abort_flag = 0;
@@ -191,36 +201,43 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t id_pv = make_idesc(kFp8 ? 0 : 1, kFp8 ? 0 : 1, 128, 1);
     const uint32_t tS[2] = {tmem + 0, tmem + 128};
     const uint32_t tO[2] = {tmem + 256, tmem + 384};
-    const uint32_t q_addr = smem_u32(sq), k_addr = smem_u32(sk), v_addr = smem_u32(sv);
+    // Descriptors are built once; the 14-bit start-address field holds
+    // (address >> 4), so moving to another tile, stage or K step is a plain
+    // add of (byte offset >> 4) (shared addresses stay below 256 KB, so the
+    // field never carries).  Built by every lane (warp-uniform values), one
+    // elected lane issues.
+    const uint64_t dq0 = make_sdesc_sw128(smem_u32(sq), 16, 1024);
+    const uint64_t dk0 = make_sdesc_sw128(smem_u32(sk), 16, 1024);
+    const uint64_t dv0 = make_sdesc_sw128(smem_u32(sv), 16384, 1024);
+    constexpr uint32_t kTileStep = C::kTile >> 4;
     auto issue_s = [&](int i, int st) {
+      const uint64_t dq = dq0 + static_cast<uint64_t>(i * kTileStep);
+      const uint64_t dk = dk0 + static_cast<uint64_t>(st * kTileStep);
       if (leader) {
 #pragma unroll
         for (int kk = 0; kk < C::kKSteps; ++kk) {
           // K-major 128B-swizzled operands: 32 bytes of K per MMA; bf16 tiles
           // hold two 64-column halves 16 KB apart
-          const uint32_t koff = kFp8 ? 32 * kk : (kk / 4) * 16384 + 32 * (kk % 4);
-          const uint64_t ad = make_sdesc_sw128(q_addr + i * C::kTile + koff, 16, 1024);
-          const uint64_t bd = make_sdesc_sw128(k_addr + st * C::kTile + koff, 16, 1024);
-          if (kFp8) mma_f8_ss(tS[i], ad, bd, id_qk, kk > 0);
-          else mma_bf16_ss(tS[i], ad, bd, id_qk, kk > 0);
+          const uint32_t koff = (kFp8 ? 32 * kk : (kk / 4) * 16384 + 32 * (kk % 4)) >> 4;
+          if (kFp8) mma_f8_ss(tS[i], dq + koff, dk + koff, id_qk, kk > 0);
+          else mma_bf16_ss(tS[i], dq + koff, dk + koff, id_qk, kk > 0);
         }
         mma_commit(&bars.s_full[i]);
       }
-      __syncwarp();
     };
     auto issue_pv = [&](int i, int st, int j) {
+      const uint64_t dv = dv0 + static_cast<uint64_t>(st * kTileStep);
+      const uint32_t acc0 = j > 0 ? 1u : 0u;
       if (leader) {
 #pragma unroll
         for (int kk = 0; kk < C::kKSteps; ++kk) {
           // V is MN-major: K (keys) advances by 32 (fp8) or 16 (bf16) rows of
           // 128 bytes; the second 64-column half of a bf16 tile sits 16 KB on
-          const uint32_t voff = kFp8 ? 4096 * kk : 2048 * kk;
-          const uint64_t bd = make_sdesc_sw128(v_addr + st * C::kTile + voff, 16384, 1024);
-          if (kFp8) mma_f8_ts(tO[i], tS[i] + 8 * kk, bd, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
-          else mma_bf16_ts(tO[i], tS[i] + 8 * kk, bd, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t voff = (kFp8 ? 4096 * kk : 2048 * kk) >> 4;
+          if (kFp8) mma_f8_ts(tO[i], tS[i] + 8 * kk, dv + voff, id_pv, kk > 0 ? 1u : acc0);
+          else mma_bf16_ts(tO[i], tS[i] + 8 * kk, dv + voff, id_pv, kk > 0 ? 1u : acc0);
         }
       }
-      __syncwarp();
     };
     bool ok = mbar_wait(&bars.q_full, 0, abort_flag) && mbar_wait(&bars.k_full[0], 0, abort_flag);
     if (ok) {
@@ -250,7 +267,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           mma_commit(&bars.kv_empty[st]);
           if (j + 1 == nkv) mma_commit(&bars.o_done[1]);
         }
-        __syncwarp();
         if (j + 1 < nkv) issue_s(1, st1);
       }
     }
@@ -278,6 +294,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float l_run = 0.0f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
+      if (kAlternate) {
+        // wait for the other warpgroup's turn to end
+        if (wg == 0 && j > 0 && !mbar_wait(&bars.tok[0], (j - 1) & 1, abort_flag)) { ok = false; break; }
+        if (wg == 1 && !mbar_wait(&bars.tok[1], j & 1, abort_flag)) { ok = false; break; }
+      }
       if (!mbar_wait(&bars.s_full[wg], j & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       uint32_t u[128];
@@ -316,8 +337,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         float t0, t1;
         f2_unpack(t, t0, t1);
         uint64_t e;
-        if ((k & 7) >= 5) {
-          // 3 of every 8 pairs on the FMA pipe, the rest on the MUFU
+        if ((k & 7) >= 8 - kPolyPairsPer8) {
+          // kPolyPairsPer8 of every 8 pairs on the FMA pipe, the rest on the MUFU
           e = f2_exp2_poly(f2_pack(fmaxf(t0, -126.0f), fmaxf(t1, -126.0f)));
         } else {
           e = f2_pack(ex2_approx(t0), ex2_approx(t1));
@@ -347,26 +368,32 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (!kFp8) tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pw[32]));
       // O_i is stable here (PV_i(j-1) finished before S_i(j) was written)
       if (j > 0 && __any_sync(0xFFFFFFFFu, m_new > m_run)) {
+        const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * c, o);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t o[64];
+          tmem_ld32(tO + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+          tmem_ld32(tO + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
           tmem_ld_wait();
-          const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-          for (int x = 0; x < 32; x += 2) {
+          for (int x = 0; x < 64; x += 2) {
             float o0, o1;
             f2_unpack(f2_mul(f2_pack(__uint_as_float(o[x]), __uint_as_float(o[x + 1])), a2), o0, o1);
             o[x] = __float_as_uint(o0);
             o[x + 1] = __float_as_uint(o1);
           }
-          tmem_st32(tO + 32 * c, o);
+          tmem_st32(tO + 64 * half, *reinterpret_cast<const uint32_t(*)[32]>(&o[0]));
+          tmem_st32(tO + 64 * half + 32, *reinterpret_cast<const uint32_t(*)[32]>(&o[32]));
         }
       }
       m_run = m_new;
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bars.p_full[wg]);
+      if (kAlternate) {
+        if (wg == 0) mbar_arrive(&bars.tok[1]);
+        else if (j + 1 < nkv) mbar_arrive(&bars.tok[0]);
+      }
     }
     if (!ok) {
       if (lane == 0) note_error(p, bars, kErrTimeout);
