@@ -228,6 +228,45 @@ int fp8attn_select_mode(const fp8attn_ctx* ctx, const uint8_t* skip_mask, int la
 fp8attn_status fp8attn_e4m3_encode(const float* d_in, int64_t n, float scale, void* d_out,
                                    void* stream);
 
+/* Allocation-free one-shot dynamic quantisation.  The pages have no
+ * counterpart to this entry point; it exists for callers that cannot
+ * allocate device memory -- for example an operator that an inference
+ * runtime hands only its input and output buffers under a fixed memory
+ * plan, or code that must not call cudaMalloc/cudaFree because those calls
+ * synchronise the device -- and so cannot provide the context workspace of
+ * fp8attn_quantize_qkv.
+ *
+ * It performs the fused amax + scale + E4M3 cast + unpad of Q, K and V in
+ * one launch, with the scales taken from this call's amax alone (no ring;
+ * identical to the first DYNAMIC pass of a freshly created context), and
+ * writes {ds_q, ds_k, ds_v} to d_descale_out (device float[3]) and, if
+ * d_scale_out is not NULL, {qs_q, qs_k, qs_v} to it.  All other arguments
+ * and layouts are those of fp8attn_quantize_qkv.
+ *
+ * Scratch: a library-owned, file-scope device array of 16,640 bytes holding
+ * one partial maximum per CTA (up to 1,024 CTAs) and the grid-barrier and
+ * error words; every GPU that loads the library holds one until the process
+ * exits.  A launch that would need more than 1,024 CTAs is refused with
+ * FP8ATTN_ERR_UNSUPPORTED (on B200 the launch uses at most 148 x 4).  The
+ * call performs no allocation of any kind.  The first call on a device looks
+ * up the array's device address (once per device); make that first call
+ * before any stream capture.  All calls share the one array, so calls whose
+ * kernels overlap on the GPU (different streams, or concurrent graphs) race
+ * and give wrong results: serialise them.  Device-side errors accumulate in
+ * the array until read with fp8attn_quantize_qkv_noalloc_error().
+ * Returns an fp8attn_status. */
+int fp8attn_quantize_qkv_noalloc(const void* q, const void* k, const void* v, int64_t tok_stride,
+                                 int64_t head_stride, const int32_t* d_src_seq_start,
+                                 const int32_t* d_cu_seqlens, int batch, int max_seqlen,
+                                 int64_t total_tokens, int num_heads, int head_dim, void* q8,
+                                 void* k8, void* v8, float* d_descale_out, float* d_scale_out,
+                                 void* stream);
+
+/* Read and clear the device-side error word of the allocation-free entry
+ * point for the current device (synchronises `stream`); after a TIMEOUT the
+ * barrier words are reset too.  Returns an fp8attn_status. */
+int fp8attn_quantize_qkv_noalloc_error(void* stream);
+
 /* Number of kernels the library has launched in this process (a counter
  * incremented on every successful launch; for accounting in benchmarks). */
 uint64_t fp8attn_launch_count(void);

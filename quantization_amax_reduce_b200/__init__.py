@@ -27,6 +27,7 @@ __all__ = [
     "DYNAMIC", "STATIC", "SKIP", "RING_LENGTH", "DEFAULT_MARGIN", "FP8AttnError", "lib",
     "Context", "varlen_fwd", "varlen_fwd_bf16", "parse_selector", "e4m3_encode",
     "launch_count", "load_scale_file", "save_scale_file", "read_error_word",
+    "quantize_qkv_noalloc", "quantize_qkv_noalloc_error",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -90,6 +91,9 @@ def lib() -> ctypes.CDLL:
         "fp8attn_select_mode": (I, [P, U8P, I]),
         "fp8attn_e4m3_encode": (I, [P, I64, F, P, P]),
         "fp8attn_launch_count": (ctypes.c_uint64, []),
+        "fp8attn_quantize_qkv_noalloc": (I, [P, P, P, I64, I64, P, P, I, I, I64, I, I, P, P, P, P,
+                                             P, P]),
+        "fp8attn_quantize_qkv_noalloc_error": (I, [P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -371,6 +375,54 @@ def e4m3_encode(x: torch.Tensor, scale: float = 1.0, stream=None) -> torch.Tenso
                                      ctypes.c_void_p(_stream(stream, x.device))),
            "fp8attn_e4m3_encode")
     return out
+
+
+def quantize_qkv_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens,
+                         max_seqlen: int, q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor,
+                         descale_out: torch.Tensor, scale_out: Optional[torch.Tensor] = None, *,
+                         total_tokens: Optional[int] = None, src_seq_start=None,
+                         stream=None) -> None:
+    """Allocation-free one-shot dynamic quantisation (scales from this call's
+    amax; no context, no workspace).  For callers that cannot allocate device
+    memory: every buffer, including the outputs ``q8``/``k8``/``v8`` and the
+    3-float ``descale_out`` (and optional ``scale_out``), is the caller's, and
+    the library keeps its reduction scratch in a fixed device array.  Calls
+    that overlap on the GPU race on that array."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _require_cuda(t, name)
+        if t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} must be bfloat16")
+    if q.stride() != k.stride() or q.stride() != v.stride() or q.shape[-1] != HEAD_DIM:
+        raise ValueError("q, k, v must share strides and have head_dim 128")
+    for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        _require_cuda(t, name)
+        if t.dtype != torch.uint8 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous uint8 tensor")
+    _require_cuda(descale_out, "descale_out")
+    if descale_out.dtype != torch.float32 or descale_out.numel() < 3:
+        raise ValueError("descale_out must hold 3 fp32 values")
+    if scale_out is not None:
+        _require_cuda(scale_out, "scale_out")
+        if scale_out.dtype != torch.float32 or scale_out.numel() < 3:
+            raise ValueError("scale_out must hold 3 fp32 values")
+    H = q.shape[-2]
+    cu = _cu_tensor(cu_seqlens, q.device)
+    if total_tokens is None:
+        if src_seq_start is not None:
+            raise ValueError("total_tokens is required with a padded source")
+        total_tokens = q.shape[-3] if q.dim() == 3 else q.shape[0] * q.shape[1]
+    sss = None if src_seq_start is None else _cu_tensor(src_seq_start, q.device)
+    _check(lib().fp8attn_quantize_qkv_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), q.stride(-3), q.stride(-2), _ptr(sss), _ptr(cu),
+        cu.numel() - 1, int(max_seqlen), int(total_tokens), H, HEAD_DIM, _ptr(q8), _ptr(k8),
+        _ptr(v8), _ptr(descale_out), _ptr(scale_out),
+        ctypes.c_void_p(_stream(stream, q.device))), "fp8attn_quantize_qkv_noalloc")
+
+
+def quantize_qkv_noalloc_error(stream=None) -> int:
+    """Read and clear the allocation-free entry point's device error word."""
+    return int(lib().fp8attn_quantize_qkv_noalloc_error(
+        ctypes.c_void_p(_stream(stream, torch.cuda.current_device()))))
 
 
 def launch_count() -> int:

@@ -393,3 +393,241 @@ cudaError_t launch_encode(const float* in, int64_t n, float scale, void* out,
 }
 
 }  // namespace fp8attn
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of the fused dynamic quantisation.
+//
+// Some callers cannot allocate device memory at all: code that runs inside a
+// host-side allocator-free region (a plugin or operator that is handed only
+// its input and output buffers by an inference runtime with a fixed memory
+// plan), or a caller that must not touch cudaMalloc/cudaFree because those
+// calls synchronise the device.  They cannot provide the context workspace
+// that fp8attn_quantize_qkv uses for its grid-wide reduction, so this
+// variant keeps that scratch in a fixed array inside the library and needs
+// nothing but the inputs and outputs.  It computes this call's per-tensor
+// amax (no ring: the scales come from this call alone, as on the first
+// dynamic pass of a fresh context), casts, and writes the scales.
+// ---------------------------------------------------------------------------
+
+#include <mutex>
+
+namespace fp8attn {
+
+namespace {
+
+// One partial |x|-max slot (q, k, v, pad) per CTA, then the barrier words.
+constexpr int kNoAllocMaxCtas = 1024;
+constexpr int kNoAllocWordBar = kNoAllocMaxCtas * 4;   // bar_count
+constexpr int kNoAllocWordGen = kNoAllocWordBar + 1;   // bar_gen
+constexpr int kNoAllocWordErr = kNoAllocWordBar + 2;   // error bits
+constexpr int kNoAllocWords = kNoAllocWordBar + 64;    // 16,640 bytes
+
+// Library-owned scratch; every device that loads the library holds its own
+// copy until the process exits.  Zero at load time.
+static __device__ __align__(256) uint32_t g_noalloc_scratch[kNoAllocWords];
+
+struct NoAllocArgs {
+  QuantArgs a;             // gs / ls unused
+  uint32_t* scratch;       // device address of g_noalloc_scratch
+  float* descale_out;      // [3] ds_q, ds_k, ds_v
+  float* scale_out;        // [3] qs_q, qs_k, qs_v, or null
+};
+
+__device__ bool noalloc_barrier(uint32_t* scratch, int* s_ok) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    volatile uint32_t* gen = scratch + kNoAllocWordGen;
+    const uint32_t my_gen = *gen;
+    __threadfence();
+    const uint32_t arrived = atomicAdd(scratch + kNoAllocWordBar, 1u) + 1u;
+    int ok = 1;
+    if (arrived == gridDim.x) {
+      scratch[kNoAllocWordBar] = 0;
+      __threadfence();
+      atomicAdd(scratch + kNoAllocWordGen, 1u);
+    } else {
+      const uint64_t t0 = global_timer_ns();
+      uint32_t it = 0;
+      while (*gen == my_gen) {
+        if ((++it & 255u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) { ok = 0; break; }
+        __nanosleep(64);
+      }
+    }
+    __threadfence();
+    *s_ok = ok;
+  }
+  __syncthreads();
+  return *s_ok != 0;
+}
+
+template <bool kContig>
+__global__ void __launch_bounds__(kThreads) quant_noalloc_kernel(NoAllocArgs n) {
+  __shared__ uint32_t red[kThreads / 32];
+  __shared__ int s_ok;
+  __shared__ float s_scale[2][3];
+  const QuantArgs& a = n.a;
+  uint32_t* scratch = n.scratch;
+  if (!seqlens_ok(a)) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(scratch + kNoAllocWordErr, kErrSeqlens);
+    return;
+  }
+  const int64_t T = __ldg(a.cu + a.B);
+  const int64_t nvec = T * a.H * 16;
+  for (int t = 0; t < 3; ++t) {
+    uint32_t m = amax_sweep<kContig>(a, t, nvec);
+    m = block_max(m, red);
+    // each CTA owns its slot and rewrites it on every call: nothing to clear
+    if (threadIdx.x == 0) scratch[blockIdx.x * 4 + t] = m;
+    if (!noalloc_barrier(scratch, &s_ok)) {
+      if (threadIdx.x == 0) atomicOr(scratch + kNoAllocWordErr, kErrTimeout);
+      return;
+    }
+    // every CTA reduces all slots the same way and gets the same bound
+    uint32_t all = 0;
+    for (uint32_t c = threadIdx.x; c < gridDim.x; c += blockDim.x)
+      all = max(all, *reinterpret_cast<volatile uint32_t*>(scratch + c * 4 + t));
+    all = block_max(all, red);
+    if (threadIdx.x == 0) {
+      const bool finite = all < 0x7F80u;
+      float qs, ds;
+      scales_from_bound(finite ? __uint_as_float(all << 16) : 0.0f, &qs, &ds);
+      s_scale[0][t] = qs;
+      s_scale[1][t] = ds;
+      if (!finite && blockIdx.x == 0) atomicOr(scratch + kNoAllocWordErr, kErrNonfinite);
+    }
+    __syncthreads();
+    cast_sweep<kContig>(a, t, nvec, s_scale[0][t], true);
+  }
+  if (blockIdx.x == 0 && threadIdx.x < 3) {
+    n.descale_out[threadIdx.x] = s_scale[1][threadIdx.x];
+    if (n.scale_out) n.scale_out[threadIdx.x] = s_scale[0][threadIdx.x];
+  }
+}
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+// Device address of the scratch array for the current device, looked up once
+// per device (host code cannot use the array's name as a device address).
+cudaError_t noalloc_scratch(uint32_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = static_cast<uint32_t*>(g_noalloc_ptr[dev]);
+  return cudaSuccess;
+}
+
+}  // namespace
+
+}  // namespace fp8attn
+
+extern "C" {
+
+// See include/fp8attn.h.
+int fp8attn_quantize_qkv_noalloc(const void* q, const void* k, const void* v, int64_t tok_stride,
+                                 int64_t head_stride, const int32_t* d_src_seq_start,
+                                 const int32_t* d_cu_seqlens, int batch, int max_seqlen,
+                                 int64_t total_tokens, int num_heads, int head_dim, void* q8,
+                                 void* k8, void* v8, float* d_descale_out, float* d_scale_out,
+                                 void* stream) {
+  using namespace fp8attn;
+  auto aligned = [](const void* p, uintptr_t al) {
+    return (reinterpret_cast<uintptr_t>(p) & (al - 1)) == 0;
+  };
+  if (batch < 1 || max_seqlen < 0 || num_heads < 1 || total_tokens < 0 || !d_cu_seqlens ||
+      !d_descale_out)
+    return 1;   // FP8ATTN_ERR_INVALID
+  if (head_dim != kHeadDim) return 4;   // FP8ATTN_ERR_UNSUPPORTED
+  if (total_tokens > static_cast<int64_t>(batch) * max_seqlen) return 1;
+  if (!q || !k || !v || !q8 || !k8 || !v8) return 1;
+  if (tok_stride <= 0 || head_stride <= 0 || (tok_stride % 8) || (head_stride % 8)) return 4;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(q8, 16) ||
+      !aligned(k8, 16) || !aligned(v8, 16) || !aligned(d_descale_out, 4) ||
+      (d_scale_out && !aligned(d_scale_out, 4)))
+    return 4;
+  uint32_t* scratch = nullptr;
+  if (noalloc_scratch(&scratch) != cudaSuccess) return 2;   // FP8ATTN_ERR_CUDA
+  NoAllocArgs n;
+  QuantArgs& a = n.a;
+  a.src[0] = static_cast<const uint16_t*>(q);
+  a.src[1] = static_cast<const uint16_t*>(k);
+  a.src[2] = static_cast<const uint16_t*>(v);
+  a.dst[0] = static_cast<uint8_t*>(q8);
+  a.dst[1] = static_cast<uint8_t*>(k8);
+  a.dst[2] = static_cast<uint8_t*>(v8);
+  a.tok_stride = tok_stride;
+  a.head_stride = head_stride;
+  a.cu = d_cu_seqlens;
+  a.src_seq_start = d_src_seq_start;
+  a.B = batch;
+  a.H = num_heads;
+  a.max_seqlen = max_seqlen;
+  a.T = total_tokens;
+  a.gs = nullptr;
+  a.ls = nullptr;
+  n.scratch = scratch;
+  n.descale_out = d_descale_out;
+  n.scale_out = d_scale_out;
+  const bool contig = d_src_seq_start == nullptr && head_stride == kHeadDim &&
+                      tok_stride == static_cast<int64_t>(num_heads) * kHeadDim;
+  const int cap = contig ? max_coresident(quant_noalloc_kernel<true>, kThreads)
+                         : max_coresident(quant_noalloc_kernel<false>, kThreads);
+  if (cap <= 0) return 2;
+  const int64_t nvec_max = total_tokens * num_heads * 16;
+  int64_t want = (nvec_max + static_cast<int64_t>(kThreads) * kUnroll - 1) /
+                 (static_cast<int64_t>(kThreads) * kUnroll);
+  if (want < 1) want = 1;
+  const int64_t grid = want < cap ? want : cap;
+  // the array holds one partial maximum per CTA: a launch needing more CTAs
+  // than it has slots is refused
+  if (grid > kNoAllocMaxCtas) return 4;   // FP8ATTN_ERR_UNSUPPORTED
+  void* args[] = {&n};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const void* fn = contig ? reinterpret_cast<const void*>(&quant_noalloc_kernel<true>)
+                          : reinterpret_cast<const void*>(&quant_noalloc_kernel<false>);
+  if (cudaLaunchKernelExC(&cfg, fn, args) != cudaSuccess) return 2;
+  return 0;
+}
+
+// See include/fp8attn.h.
+int fp8attn_quantize_qkv_noalloc_error(void* stream) {
+  using namespace fp8attn;
+  uint32_t* scratch = nullptr;
+  if (noalloc_scratch(&scratch) != cudaSuccess) return 2;
+  uint32_t bits = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(&bits, scratch + kNoAllocWordErr, sizeof(bits),
+                                  cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return 2;
+  if (bits) {
+    // clear the error; after a timeout also reset the barrier words
+    e = cudaMemsetAsync(scratch + kNoAllocWordBar, 0,
+                        (bits & kErrTimeout) ? 3 * sizeof(uint32_t) : 0, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(scratch + kNoAllocWordErr, 0, sizeof(uint32_t), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return 2;
+  }
+  if (bits & kErrTimeout) return 3;
+  if (bits & kErrSeqlens) return 6;
+  if (bits & kErrNonfinite) return 5;
+  return 0;
+}
+
+}  // extern "C"
