@@ -210,34 +210,49 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint64_t dk0 = make_sdesc_sw128(smem_u32(sk), 16, 1024);
     const uint64_t dv0 = make_sdesc_sw128(smem_u32(sv), 16384, 1024);
     constexpr uint32_t kTileStep = C::kTile >> 4;
+    // Every lane builds the descriptors of a group (warp-uniform values, so
+    // they can live in uniform registers); one elected lane then issues the
+    // MMAs back to back with nothing else in between.
     auto issue_s = [&](int i, int st) {
+      uint64_t ad[C::kKSteps], bd[C::kKSteps];
       const uint64_t dq = dq0 + static_cast<uint64_t>(i * kTileStep);
       const uint64_t dk = dk0 + static_cast<uint64_t>(st * kTileStep);
-      if (leader) {
+#pragma unroll
+      for (int kk = 0; kk < C::kKSteps; ++kk) {
+        // K-major 128B-swizzled operands: 32 bytes of K per MMA; bf16 tiles
+        // hold two 64-column halves 16 KB apart
+        const uint32_t koff = (kFp8 ? 32 * kk : (kk / 4) * 16384 + 32 * (kk % 4)) >> 4;
+        ad[kk] = dq + koff;
+        bd[kk] = dk + koff;
+      }
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < C::kKSteps; ++kk) {
-          // K-major 128B-swizzled operands: 32 bytes of K per MMA; bf16 tiles
-          // hold two 64-column halves 16 KB apart
-          const uint32_t koff = (kFp8 ? 32 * kk : (kk / 4) * 16384 + 32 * (kk % 4)) >> 4;
-          if (kFp8) mma_f8_ss(tS[i], dq + koff, dk + koff, id_qk, kk > 0);
-          else mma_bf16_ss(tS[i], dq + koff, dk + koff, id_qk, kk > 0);
+          if (kFp8) mma_f8_ss(tS[i], ad[kk], bd[kk], id_qk, kk > 0);
+          else mma_bf16_ss(tS[i], ad[kk], bd[kk], id_qk, kk > 0);
         }
         mma_commit(&bars.s_full[i]);
       }
+      __syncwarp();
     };
     auto issue_pv = [&](int i, int st, int j) {
+      uint64_t bd[C::kKSteps];
       const uint64_t dv = dv0 + static_cast<uint64_t>(st * kTileStep);
+#pragma unroll
+      for (int kk = 0; kk < C::kKSteps; ++kk) {
+        // V is MN-major: K (keys) advances by 32 (fp8) or 16 (bf16) rows of
+        // 128 bytes; the second 64-column half of a bf16 tile sits 16 KB on
+        bd[kk] = dv + ((kFp8 ? 4096 * kk : 2048 * kk) >> 4);
+      }
       const uint32_t acc0 = j > 0 ? 1u : 0u;
-      if (leader) {
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < C::kKSteps; ++kk) {
-          // V is MN-major: K (keys) advances by 32 (fp8) or 16 (bf16) rows of
-          // 128 bytes; the second 64-column half of a bf16 tile sits 16 KB on
-          const uint32_t voff = (kFp8 ? 4096 * kk : 2048 * kk) >> 4;
-          if (kFp8) mma_f8_ts(tO[i], tS[i] + 8 * kk, dv + voff, id_pv, kk > 0 ? 1u : acc0);
-          else mma_bf16_ts(tO[i], tS[i] + 8 * kk, dv + voff, id_pv, kk > 0 ? 1u : acc0);
+          if (kFp8) mma_f8_ts(tO[i], tS[i] + 8 * kk, bd[kk], id_pv, kk > 0 ? 1u : acc0);
+          else mma_bf16_ts(tO[i], tS[i] + 8 * kk, bd[kk], id_pv, kk > 0 ? 1u : acc0);
         }
       }
+      __syncwarp();
     };
     bool ok = mbar_wait(&bars.q_full, 0, abort_flag) && mbar_wait(&bars.k_full[0], 0, abort_flag);
     if (ok) {
@@ -252,7 +267,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!ok) break;
         tc_fence_after();
         issue_pv(0, st, j);
-        if (j + 1 == nkv && leader) mma_commit(&bars.o_done[0]);
+        if (j + 1 == nkv) {
+          if (elect_one()) mma_commit(&bars.o_done[0]);
+          __syncwarp();
+        }
         if (j + 1 < nkv) {
           ok = mbar_wait(&bars.k_full[st1], ((j + 1) / C::kStages) & 1, abort_flag);
           if (!ok) break;
@@ -263,16 +281,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!ok) break;
         tc_fence_after();
         issue_pv(1, st, j);
-        if (leader) {
+        if (elect_one()) {
           mma_commit(&bars.kv_empty[st]);
           if (j + 1 == nkv) mma_commit(&bars.o_done[1]);
         }
+        __syncwarp();
         if (j + 1 < nkv) issue_s(1, st1);
       }
     }
     if (!ok && leader) note_error(p, bars, kErrTimeout);
-    // drain: every MMA this thread issued has completed before TMEM is freed
-    if (leader) mma_commit(&bars.drain);
+    // drain: every MMA this warp issued has completed before TMEM is freed
+    if (elect_one()) mma_commit(&bars.drain);
     __syncwarp();
     mbar_wait(&bars.drain, 0, nullptr);
   } else {

@@ -77,19 +77,33 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that lets the hardware suspend the thread until the phase
+// completes or `suspend_ns` elapses, so waiting warps take no issue slots.
+__device__ __forceinline__ bool mbar_test_suspend(uint64_t* bar, uint32_t parity,
+                                                  uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with the given parity has completed.  Returns false
 // if the wait ran past kWaitLimitNs or `abort_flag` (shared memory, may be
-// null) became non-zero.
+// null) became non-zero.  Each try suspends the thread for at most 0.2 ms,
+// so the limit and the abort flag are checked regularly.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           const volatile int* abort_flag) {
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_test(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (abort_flag && *abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) return false;
-    }
+  for (;;) {
+    if (mbar_test_suspend(bar, parity, 200000u)) return true;
+    if (abort_flag && *abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
   }
 }
 
