@@ -94,16 +94,19 @@ __device__ __forceinline__ bool mbar_test_suspend(uint64_t* bar, uint32_t parity
 
 // Wait until the phase with the given parity has completed.  Returns false
 // if the wait ran past kWaitLimitNs or `abort_flag` (shared memory, may be
-// null) became non-zero.  Each try suspends the thread for at most 0.2 ms,
-// so the limit and the abort flag are checked regularly.
+// null) became non-zero.  Spins on try_wait (no suspend hint: a suspended
+// thread can wake well after the phase completes); the limit and the abort
+// flag are checked every 64 tries.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           const volatile int* abort_flag) {
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (;;) {
-    if (mbar_test_suspend(bar, parity, 200000u)) return true;
-    if (abort_flag && *abort_flag) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_test(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (abort_flag && *abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    }
   }
 }
 

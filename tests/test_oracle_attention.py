@@ -156,8 +156,8 @@ def test_row_subset_equals_full_rows():
 
 def test_pquant_rule_uses_running_block_max():
     # 129 keys: keys 0..127 score 0 (block 0), key 128 scores 1 (block 1).
-    # Block 0 is quantised against its own max 0: p = 1 -> 256 is exact, then
-    # carried to the final max 1 by the exact factor e^-1, so p~ = e^-1.
+    # Block 0 is quantised against its running max 0: p = 1 -> 256 is exact,
+    # then carried to the final max 1 by the exact factor e^-1, so p~ = e^-1.
     # (Against the final max it would be e4m3(256 e^-1) = e4m3(94.18) = 96,
     # p~ = 0.375.)  Key 128: p~ = 1.  l = 128 e^-1 + 1 (unquantised).
     D, n = 128, 129
@@ -175,6 +175,25 @@ def test_pquant_rule_uses_running_block_max():
     assert abs(o[0, 0, 1] - 1.0 / l) < 1e-15
     assert abs(o[0, 0, 2] - math.exp(-1.0) / l) < 1e-15
     assert abs(o[0, 0, 2] - 0.375 / l) > 1e-4       # not the final-max rule
+
+
+def test_pquant_block_is_128_keys():
+    # keys 0..63 score 0, key 64 scores 1: all in block 0 (128 keys), so
+    # keys 0..63 are quantised against the block max 1, giving
+    # e4m3(256 e^-1)/256 = 96/256 = 0.375 (with 64-key blocks they would be
+    # quantised against max 0 and give e^-1 exactly).
+    D, n = 128, 65
+    q8 = np.zeros((n, 1, D), np.uint8)
+    k8 = np.zeros((n, 1, D), np.uint8)
+    v8 = np.zeros((n, 1, D), np.uint8)
+    q8[:, 0, 0] = 0x38
+    k8[64, 0, 0] = 0x38               # s_64 = 1
+    v8[0, 0, 2] = 0x38                # v_0 = e_2
+    cu = np.array([0, n], dtype=np.int32)
+    o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True,
+                             rows=[0])
+    l = 64 * math.exp(-1.0) + 1.0
+    assert abs(o[0, 0, 2] - 0.375 / l) < 1e-15
 
 
 def test_pquant_block_rule_second_block_lower_max():
