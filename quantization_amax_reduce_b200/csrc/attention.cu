@@ -84,7 +84,8 @@ struct Barriers {
   int abort_flag;
 };
 
-__device__ __forceinline__ void note_error(AttnParams& p, Barriers& bars, uint32_t bit) {
+template <typename Bars>
+__device__ __forceinline__ void note_error(AttnParams& p, Bars& bars, uint32_t bit) {
   bars.abort_flag = 1;
   if (p.err) atomicOr(reinterpret_cast<unsigned int*>(p.err), bit);
 }
@@ -455,6 +456,370 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
+
+// ---------------------------------------------------------------------------
+// FP8 path with P in shared memory.
+//
+// The softmax of query tile i hands its S columns back to the MMA warp as
+// soon as it has loaded block j into registers (s_free), so S_i(j+1) is
+// computed while the softmax is still working on block j: the softmax of
+// consecutive key blocks runs back to back instead of waiting for its own
+// PV and S round trip.  P_i(j) goes to a swizzled shared-memory buffer
+// (double-buffered per tile) that the PV MMA reads as its K-major A operand.
+// Ordering facts used below (MMAs of one thread complete in issue order):
+//   - S_i(j+1) is issued after PV_i(j-1), so when the softmax sees S_i(j+1)
+//     complete, PV_i(j-1) (and the P buffer it read) is done;
+//   - the O rescale of block j needs PV_i(j-1): it waits on the P buffer's
+//     barrier, which is at most one phase behind.
+// ---------------------------------------------------------------------------
+
+struct Fp8Cfg {
+  static constexpr int kStages = 3;
+  static constexpr int kTile = 16384;   // 128 x 128 bytes
+  static constexpr int kSmemBytes = (2 + 2 * kStages + 4) * kTile + 1024 + 1024;
+};
+
+struct Fp8Barriers {
+  uint64_t q_full;
+  uint64_t k_full[Fp8Cfg::kStages];
+  uint64_t v_full[Fp8Cfg::kStages];
+  uint64_t kv_empty[Fp8Cfg::kStages];
+  uint64_t s_full[2];       // S_i of the current block computed
+  uint64_t s_free[2];       // S_i loaded by the softmax (TMEM columns free)
+  uint64_t p_full[2][2];    // [tile][P buffer] P_i written
+  uint64_t pv_done[2][2];   // [tile][P buffer] PV_i that read that buffer done
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__global__ void __launch_bounds__(kThreadsAttn, 1)
+attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, AttnParams p) {
+  using C = Fp8Cfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sq = smem;                                   // 2 Q tiles
+  uint8_t* sk = smem + 2 * C::kTile;                    // kStages K tiles
+  uint8_t* sv = sk + C::kStages * C::kTile;             // kStages V tiles
+  uint8_t* sp = sv + C::kStages * C::kTile;             // P [tile][buffer]
+  Fp8Barriers& bars = *reinterpret_cast<Fp8Barriers*>(sp + 4 * C::kTile);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int qb = blockIdx.x % p.n_qblk;
+  const int bh = blockIdx.x / p.n_qblk;
+  const int h = bh % p.H;
+  const int b = bh / p.H;
+  const int seq0 = __ldg(p.cu + b);
+  const int seq1 = __ldg(p.cu + b + 1);
+  const int len = seq1 - seq0;
+  if (seq0 < 0 || len < 0 || len > p.max_seqlen || static_cast<int64_t>(seq1) > p.T) {
+    if (threadIdx.x == 0 && qb == 0 && p.err)
+      atomicOr(reinterpret_cast<unsigned int*>(p.err), kErrSeqlens);
+    return;
+  }
+  const int q0 = qb * 256;
+  if (q0 >= len) return;
+  const int nkv = (len + 127) / 128;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars.q_full, 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&bars.k_full[s], 1);
+      mbar_init(&bars.v_full[s], 1);
+      mbar_init(&bars.kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.s_full[i], 1);
+      mbar_init(&bars.s_free[i], 128);
+      for (int q = 0; q < 2; ++q) {
+        mbar_init(&bars.p_full[i][q], 128);
+        mbar_init(&bars.pv_done[i][q], 1);
+      }
+    }
+    mbar_init(&bars.drain, 1);
+    bars.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&bars.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars.tmem_base;
+  const volatile int* abort_flag = &bars.abort_flag;
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ producer
+    const bool leader = lane == 0;
+    if (leader) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_expect_tx(&bars.q_full, 2 * C::kTile);
+      for (int i = 0; i < 2; ++i)
+        tma_load_3d(sq + i * C::kTile, &tm_q, &bars.q_full, 0, h, seq0 + q0 + 128 * i);
+    }
+    int issued = 0;
+    for (int j = 0; j < nkv; ++j) {
+      const int st = j % C::kStages;
+      if (j >= C::kStages) {
+        if (!mbar_wait(&bars.kv_empty[st], ((j / C::kStages) - 1) & 1, abort_flag)) {
+          if (leader) note_error(p, bars, kErrTimeout);
+          break;
+        }
+      }
+      if (leader) {
+        const int tok = seq0 + 128 * j;
+        mbar_expect_tx(&bars.k_full[st], C::kTile);
+        tma_load_3d(sk + st * C::kTile, &tm_k, &bars.k_full[st], 0, h, tok);
+        mbar_expect_tx(&bars.v_full[st], C::kTile);
+        tma_load_3d(sv + st * C::kTile, &tm_v, &bars.v_full[st], 0, h, tok);
+      }
+      __syncwarp();
+      issued = j + 1;
+    }
+    for (int j = (issued > C::kStages ? issued - C::kStages : 0); j < issued; ++j) {
+      const int st = j % C::kStages;
+      mbar_wait(&bars.k_full[st], (j / C::kStages) & 1, nullptr);
+      mbar_wait(&bars.v_full[st], (j / C::kStages) & 1, nullptr);
+    }
+    mbar_wait(&bars.q_full, 0, nullptr);
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    const bool leader = lane == 0;
+    const uint32_t id_qk = make_idesc(0, 0, 128, 0);
+    const uint32_t id_pv = make_idesc(0, 0, 128, 1);
+    const uint64_t dq0 = make_sdesc_sw128(smem_u32(sq), 16, 1024);
+    const uint64_t dk0 = make_sdesc_sw128(smem_u32(sk), 16, 1024);
+    const uint64_t dv0 = make_sdesc_sw128(smem_u32(sv), 16384, 1024);
+    const uint64_t dp0 = make_sdesc_sw128(smem_u32(sp), 16, 1024);
+    constexpr uint32_t kStep = C::kTile >> 4;
+    auto issue_s = [&](int i, int j) {
+      uint64_t ad[4], bd[4];
+      const uint64_t dq = dq0 + static_cast<uint64_t>(i * kStep);
+      const uint64_t dk = dk0 + static_cast<uint64_t>((j % C::kStages) * kStep);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        ad[kk] = dq + 2 * kk;   // 32 bytes of K per MMA
+        bd[kk] = dk + 2 * kk;
+      }
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tmem + 128 * i, ad[kk], bd[kk], id_qk, kk > 0);
+        mma_commit(&bars.s_full[i]);
+      }
+      __syncwarp();
+    };
+    auto issue_pv = [&](int i, int j) {
+      uint64_t ad[4], bd[4];
+      const uint64_t dp = dp0 + static_cast<uint64_t>((2 * i + (j & 1)) * kStep);
+      const uint64_t dv = dv0 + static_cast<uint64_t>((j % C::kStages) * kStep);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        ad[kk] = dp + 2 * kk;          // P is K-major: 32 keys per MMA
+        bd[kk] = dv + 256 * kk;        // V is MN-major: 32 rows of 128 bytes per MMA
+      }
+      const uint32_t acc0 = j > 0 ? 1u : 0u;
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f8_ss(tmem + 256 + 128 * i, ad[kk], bd[kk], id_pv, kk > 0 ? 1u : acc0);
+        mma_commit(&bars.pv_done[i][j & 1]);
+      }
+      __syncwarp();
+    };
+    bool ok = mbar_wait(&bars.q_full, 0, abort_flag) && mbar_wait(&bars.k_full[0], 0, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      issue_s(0, 0);
+      issue_s(1, 0);
+    }
+    for (int j = 0; j < nkv && ok; ++j) {
+      const int st = j % C::kStages;
+      if (j + 1 < nkv) {
+        const int st1 = (j + 1) % C::kStages;
+        ok = mbar_wait(&bars.k_full[st1], ((j + 1) / C::kStages) & 1, abort_flag);
+        for (int i = 0; i < 2 && ok; ++i) {
+          // S_i's TMEM columns are free once the softmax has loaded block j
+          ok = mbar_wait(&bars.s_free[i], j & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(i, j + 1);
+        }
+        if (!ok) break;
+      }
+      ok = mbar_wait(&bars.v_full[st], (j / C::kStages) & 1, abort_flag);
+      for (int i = 0; i < 2 && ok; ++i) {
+        ok = mbar_wait(&bars.p_full[i][j & 1], (j >> 1) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(i, j);
+      }
+      if (!ok) break;
+      if (elect_one()) mma_commit(&bars.kv_empty[st]);
+      __syncwarp();
+    }
+    if (!ok && leader) note_error(p, bars, kErrTimeout);
+    if (elect_one()) mma_commit(&bars.drain);
+    __syncwarp();
+    mbar_wait(&bars.drain, 0, nullptr);
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int wg = warp >> 2;
+    const int wq = warp & 3;
+    const int row = 32 * wq + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * wq) << 16;
+    const uint32_t tS = tmem + 128 * wg + lane_off;
+    const uint32_t tO = tmem + 256 + 128 * wg + lane_off;
+    // this row's place in the 128B-swizzled K-major P tile
+    uint8_t* prow0 = sp + (2 * wg) * C::kTile + (row >> 3) * 1024 + (row & 7) * 128;
+    const float cscale = __ldg(p.descale + 0) * __ldg(p.descale + 1) * p.softmax_scale * kLog2e;
+    const float ds_v = __ldg(p.descale + 2);
+    float m_run = -INFINITY;
+    float l_run = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      if (!mbar_wait(&bars.s_full[wg], j & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t u[128];
+      tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+      tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&u[64]));
+      tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&u[96]));
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&bars.s_free[wg]);   // the MMA warp may compute S_i(j+1) now
+      const int valid = len - 128 * j;
+      if (valid < 128) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= valid) u[c] = 0xFF800000u;   // -inf: key beyond the sequence
+      }
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; c += 8) {
+        mx0 = fmax3(mx0, __uint_as_float(u[c + 0]), __uint_as_float(u[c + 1]));
+        mx1 = fmax3(mx1, __uint_as_float(u[c + 2]), __uint_as_float(u[c + 3]));
+        mx2 = fmax3(mx2, __uint_as_float(u[c + 4]), __uint_as_float(u[c + 5]));
+        mx3 = fmax3(mx3, __uint_as_float(u[c + 6]), __uint_as_float(u[c + 7]));
+      }
+      const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3));
+      const float m_new = fmaxf(m_run, mx * cscale);
+      const float neg = 8.0f - m_new;
+      const uint64_t c2 = f2_pack(cscale, cscale);
+      const uint64_t n2 = f2_pack(neg, neg);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      uint32_t pw[32];
+#pragma unroll
+      for (int k = 0; k < 64; ++k) {
+        const uint64_t t = f2_fma(f2_pack(__uint_as_float(u[2 * k]), __uint_as_float(u[2 * k + 1])),
+                                  c2, n2);
+        float t0, t1;
+        f2_unpack(t, t0, t1);
+        uint64_t e;
+        if ((k & 7) >= 8 - kPolyPairsPer8)
+          e = f2_exp2_poly(f2_pack(fmaxf(t0, -126.0f), fmaxf(t1, -126.0f)));
+        else
+          e = f2_pack(ex2_approx(t0), ex2_approx(t1));
+        acc[k & 3] = f2_add(acc[k & 3], e);
+        float e0, e1;
+        f2_unpack(e, e0, e1);
+        const uint32_t hh = cvt_e4m3x2(e0, e1);
+        if (k & 1) pw[k >> 1] |= hh << 16;
+        else pw[k >> 1] = hh;
+      }
+      // P row -> shared memory (buffer j % 2 is free: S_i(j) complete means
+      // PV_i(j-2), its last reader, is done)
+      uint8_t* prow = prow0 + (j & 1) * C::kTile;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
+            make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+      fence_proxy_async();
+      float sum;
+      {
+        float a0, a1;
+        f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
+        sum = a0 + a1;
+      }
+      const float alpha = ex2_approx(m_run - m_new);   // 0 on the first block
+      l_run = l_run * alpha + sum;
+      if (j > 0 && __any_sync(0xFFFFFFFFu, m_new > m_run)) {
+        // O_i holds PV up to block j-1: wait for it before rescaling
+        if (!mbar_wait(&bars.pv_done[wg][(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t a2 = f2_pack(alpha, alpha);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t o[64];
+          tmem_ld32(tO + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+          tmem_ld32(tO + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+          tmem_ld_wait();
+#pragma unroll
+          for (int x = 0; x < 64; x += 2) {
+            float o0, o1;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(o[x]), __uint_as_float(o[x + 1])), a2), o0, o1);
+            o[x] = __float_as_uint(o0);
+            o[x + 1] = __float_as_uint(o1);
+          }
+          tmem_st32(tO + 64 * half, *reinterpret_cast<const uint32_t(*)[32]>(&o[0]));
+          tmem_st32(tO + 64 * half + 32, *reinterpret_cast<const uint32_t(*)[32]>(&o[32]));
+        }
+        tmem_st_wait();
+      }
+      m_run = m_new;
+      tc_fence_before();
+      mbar_arrive(&bars.p_full[wg][j & 1]);
+    }
+    if (!ok) {
+      if (lane == 0) note_error(p, bars, kErrTimeout);
+    } else if (mbar_wait(&bars.pv_done[wg][(nkv - 1) & 1], ((nkv - 1) >> 1) & 1, abort_flag)) {
+      tc_fence_after();
+      const int qrow = q0 + 128 * wg + row;
+      const bool store = qrow < len;
+      const float inv = ds_v / l_run;
+      __nv_bfloat16* dst = p.out + (static_cast<int64_t>(seq0 + qrow) * p.H + h) * kHeadDim;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * c, o);
+        tmem_ld_wait();
+        uint32_t w[16];
+        const uint64_t inv2 = f2_pack(inv, inv);
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          float o0, o1;
+          f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * x]), __uint_as_float(o[2 * x + 1])), inv2),
+                    o0, o1);
+          w[x] = cvt_bf16x2(o0, o1);
+        }
+        if (store) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) d4[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+        }
+      }
+    } else if (lane == 0) {
+      note_error(p, bars, kErrTimeout);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -496,11 +861,13 @@ cudaError_t launch_attention_t(const AttnLaunch& a, int64_t T, cudaStream_t stre
   if (!make_qkv_map(&mq, a.q, T, a.heads, !kFp8) || !make_qkv_map(&mk, a.k, T, a.heads, !kFp8) ||
       !make_qkv_map(&mv, a.v, T, a.heads, !kFp8))
     return cudaErrorInvalidValue;
+  // FP8 runs the P-in-shared-memory kernel; BF16 keeps P in TMEM
+  auto kernel = kFp8 ? attn_fwd_fp8_kernel : attn_fwd_kernel<false>;
+  const int smem_bytes = kFp8 ? Fp8Cfg::kSmemBytes : C::kSmemBytes;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<kFp8>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem_bytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -518,8 +885,7 @@ cudaError_t launch_attention_t(const AttnLaunch& a, int64_t T, cudaStream_t stre
   const int64_t grid = static_cast<int64_t>(p.n_qblk) * a.heads * a.batch;
   if (grid <= 0) return cudaSuccess;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
-  attn_fwd_kernel<kFp8><<<static_cast<unsigned>(grid), kThreadsAttn, C::kSmemBytes, stream>>>(
-      mq, mk, mv, p);
+  kernel<<<static_cast<unsigned>(grid), kThreadsAttn, smem_bytes, stream>>>(mq, mk, mv, p);
   return cudaGetLastError();
 }
 
