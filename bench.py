@@ -402,12 +402,12 @@ def run_ours(args):
             "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": fp8_peak,
                          "unit": "TFLOP/s", "frac": attn_tflops / fp8_peak,
                          "traffic": profiled_traffic(),
-                         "kernel": "attn_fwd_kernel<fp8>",
+                         "kernel": "attn_fwd_fp8_kernel",
                          "peak_source": f"{src} bf16 burst x{FP8_PER_BF16:g} (fp8/bf16 nominal)"},
             "quant_roofline": {"bound": "hbm", "achieved": quant_gbs, "peak": peaks["hbm_gbs"],
                                "unit": "GB/s", "frac": quant_gbs / peaks["hbm_gbs"],
                                "kernel": "quant_static_kernel", "peak_source": src},
-            "kernel_share": {"attn_fwd_kernel<fp8>": share_attn,
+            "kernel_share": {"attn_fwd_fp8_kernel": share_attn,
                              "quant_static_kernel": 1.0 - share_attn},
             "e2e": {"value": FLOPS_PER_STEP * E * world / e2e_max / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": 3 * S * H * D * 2, "d2h_bytes_per_step": S * H * D * 2,

@@ -10,17 +10,17 @@
 // that sequence's 128-key K/V tiles once for both:
 //   warp 8       TMA producer: Q tiles once, then a ring of K/V stages
 //   warp 9       MMA issuer (one lane): S_i = Q_i K^T into TMEM, then
-//                O_i += P_i V from TMEM (P) and shared memory (V, MN-major)
+//                O_i += P_i V (V in shared memory, MN-major)
 //   warps 0-3    softmax for query tile 0, warps 4-7 for tile 1: one thread
 //                per query row (= TMEM lane), running max, exp2 with the
 //                descales folded into one FMA, row sum of the unquantised
-//                p, P written back into the S columns, O rescaled in TMEM
-//                when the row max grows, and the bf16 epilogue.
-// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512);
-// P_i aliases the first 32 (fp8) or 64 (bf16) columns of S_i.  The MMAs of
-// one thread execute in issue order, so S_i(j+1) never overwrites P_i(j)
-// before PV_i(j) has read it, and the arrival of S_i(j+1) also means
-// PV_i(j) has finished (O_i is stable for the rescale).
+//                p, P quantised for the PV product, O rescaled in TMEM when
+//                the row max grows, and the bf16 epilogue.
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512).
+// attn_fwd_kernel (BF16): P_i aliases the first 64 columns of S_i and PV
+// reads it from TMEM; S_i(j+1) is issued after PV_i(j).
+// attn_fwd_fp8_kernel (FP8): P_i goes to shared memory, so S_i(j+1) is
+// computed while the softmax still works on block j (details there).
 //
 // P rule (pages silent; fixed here): p' = 2^(s*c - m + 8) = 256 p with c =
 // ds_q ds_k softmax_scale log2(e) and m the running max of s*c; P = e4m3(p')
