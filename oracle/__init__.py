@@ -31,8 +31,9 @@ _lib = None
 RING_LEN = 16          # vLLM FP8 ViT page: 16 observed amax values
 DEFAULT_MARGIN = 1.5   # vLLM FP8 ViT page: --mm-encoder-fp8-scale-save-margin
 E4M3_MAX = 448.0       # OCP E4M3 (FN) largest finite magnitude
-P_SCALE = 256.0        # P is quantised as e4m3(256 p) (power of two: exact)
-P_BLOCK = 128          # keys per P-quantisation block (running-max reference)
+P_SCALE = 32.0         # P is quantised as e4m3(32 exp(s - r)) (power of two: exact)
+P_BLOCK = 128          # keys per P-quantisation block
+P_LAG_LOG2 = 3.0       # the reference max r moves only when a block max exceeds it by more
 
 
 class _Ring(ctypes.Structure):
@@ -229,13 +230,17 @@ def attention_fp8(q8, k8, v8, cu, ds_qkv: Sequence[float], scale: Optional[float
     """fp64 attention on E4M3 codes [T, H, D]; returns [len(rows) or T, H, D].
 
     With ``pquant`` the PV product uses P quantised per block of 128 keys (in
-    sequence order) as e4m3(256 exp(s - m))/256, m the running row max over
-    the keys seen so far, carried exactly to the final max M; l is the sum of
-    the unquantised exp(s - M) unless ``l_of_quantized``.
+    sequence order) as e4m3(32 exp(s - r))/32 against the row's reference max
+    r: block 0's max, replaced by a later block's max only when that exceeds
+    r by more than 3 in log2 units; each block is carried exactly to the final
+    max M; l is the sum of the unquantised exp(s - M) unless
+    ``l_of_quantized``.
 
     With ``return_ambiguity`` also returns, per output, the largest change
     that P codes lying within an fp32 evaluation's error of a rounding tie
-    can make (either neighbouring code is a correct result there)."""
+    can make (either neighbouring code is a correct result there), and +inf
+    for every output of a row whose reference-max move was decided within
+    such an error of the threshold (that row cannot be compared)."""
     q8 = np.ascontiguousarray(q8, dtype=np.uint8)
     k8 = np.ascontiguousarray(k8, dtype=np.uint8)
     v8 = np.ascontiguousarray(v8, dtype=np.uint8)

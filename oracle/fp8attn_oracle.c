@@ -29,11 +29,13 @@
  *   - static values are bounds A in activation units (the margin is applied
  *     when they are saved, never again on load).
  *   - attention: P for the PV product is quantised block by block (128
- *     keys, in sequence order) as e4m3(256 exp(s - m))/256 against the
- *     running row max m over the keys seen so far -- the rule a single-pass
- *     (online-softmax) kernel applies -- and carried to the final max M
- *     exactly; the output is normalised by l = sum of the unquantised
- *     exp(s - M).
+ *     keys, in sequence order) as e4m3(32 exp(s - r))/32 against a reference
+ *     max r that a single-pass (online-softmax) kernel keeps per row: r is
+ *     the first block's max and moves to a later block's max only when that
+ *     block's max exceeds r by more than 3 in log2 units (so 32 exp(s - r)
+ *     stays at or below 2^8 = 256 and never saturates); each block's P is
+ *     carried to the final max M exactly; the output is normalised by l =
+ *     sum of the unquantised exp(s - M).
  *
  * Floating point: quantisation follows the kernel's stated fp32 rules (one
  * fp32 RN multiply, one fp32 RN division), attention is evaluated in fp64.
@@ -327,7 +329,7 @@ typedef struct {
     int B, H, D;
     double ds_q, ds_k, ds_v;
     double scale;             /* softmax scale (1/sqrt(D) by default) */
-    int pquant;               /* 0: p~ = p, 1: p~ = e4m3(256 p)/256 */
+    int pquant;               /* 0: p~ = p, 1: the block rule with a lagged reference max */
     int lrule;                /* 0: l = sum p, 1: l = sum p~ */
     const int64_t* rows;      /* token indices to evaluate (or NULL: all) */
     int64_t nrows;
@@ -345,16 +347,21 @@ static double elem(const att_job* j, const void* base, int64_t t, int h, int d) 
 
 /* P rule: the PV product takes P in blocks of OR_P_BLOCK keys, visited in
  * order from the start of the sequence; each block's p are quantised as
- * e4m3(256 exp(s - m_t)) / 256 against the running max m_t over the keys
- * seen so far (blocks 0..t), then carried to the final max M by the exact
- * factor exp(m_t - M).  l is the sum of the unquantised p = exp(s - M). */
+ * e4m3(OR_P_SCALE exp(s - r_t)) / OR_P_SCALE against the row's reference max
+ * r_t, then carried to the final max M by the exact factor exp(r_t - M).
+ * r_0 is block 0's max; r_t is block t's max when that exceeds r_{t-1} by
+ * more than OR_P_LAG_LOG2 in log2 units, else r_{t-1}.  With the lag at most
+ * 3 and the scale 2^5, OR_P_SCALE exp(s - r_t) <= 2^8 (no saturation).  l is
+ * the sum of the unquantised p = exp(s - M). */
 #define OR_P_BLOCK 128
+#define OR_P_SCALE 32.0
+#define OR_P_LAG_LOG2 3.0
 
 /* Codes within reach of a rounding tie.  An implementation evaluates
- * y = 256 exp(s - m) in fp32 (exp2 of s*log2(e) - m*log2(e) + 8), so its y
+ * y = 32 exp(s - r) in fp32 (exp2 of s*log2(e) - r*log2(e) + 5), so its y
  * carries a relative error of a few fp32 roundings of the exponent's terms
  * plus the exp2 approximation; bound it by
- *     eps(y) = 2^-20 * (2 + |s| log2(e) + |m| log2(e))
+ *     eps(y) = 2^-20 * (2 + |s| log2(e) + |r| log2(e))
  * (16x the fp32 rounding of each term).  When [y(1-eps), y(1+eps)] holds a
  * tie between two E4M3 values, either code is a correct result of the rule;
  * the caller receives the largest output change such a flip can make. */
@@ -364,14 +371,27 @@ static double code_ambiguity(double y, double s, double m) {
     uint8_t lo = or_e4m3_encode(y * (1.0 - eps));
     uint8_t hi = or_e4m3_encode(y * (1.0 + eps));
     if (lo == hi) return 0.0;
-    return fabs(or_e4m3_value(hi) - or_e4m3_value(lo)) / 256.0;
+    return fabs(or_e4m3_value(hi) - or_e4m3_value(lo)) / OR_P_SCALE;
+}
+
+/* Whether the reference max moves at a block is decided by an implementation
+ * in fp32 (a block max of fp32 scores times the scale product, against r plus
+ * the lag); when the fp64 comparison is within the same few fp32 roundings
+ * of a tie, either decision is a correct result of the rule, and every later
+ * P code of the row may differ.  Such rows are reported as unverifiable. */
+static int move_is_ambiguous(double blk_max, double r) {
+    const double log2e = 1.4426950408889634;
+    double a = blk_max * log2e, b = r * log2e + OR_P_LAG_LOG2;
+    double eps = ldexp(1.0, -18) * (4.0 + fabs(a));
+    return fabs(a - b) <= eps;
 }
 
 static void attend_one(const att_job* j, int64_t ri, int h, double* s_buf) {
     int64_t t = j->rows ? j->rows[ri] : ri;
     int b, d;
     int64_t k0, k1, kk;
-    double M = -INFINITY, l = 0.0, m_blk = -INFINITY;
+    double M = -INFINITY, l = 0.0, r = -INFINITY;
+    int unverifiable = 0;
     double* o = j->out + (ri * j->H + h) * (int64_t)j->D;
     double* a = j->amb ? j->amb + (ri * j->H + h) * (int64_t)j->D : NULL;
     double dsq = j->kind == 0 ? j->ds_q : 1.0;
@@ -396,16 +416,23 @@ static void attend_one(const att_job* j, int64_t ri, int h, double* s_buf) {
         double p = exp(s - M);
         double pt = p;
         if ((kk - k0) % OR_P_BLOCK == 0) {
-            /* entering a new block: running max over blocks seen so far */
+            /* entering a new block: its max, and whether the reference moves */
             int64_t e = kk + OR_P_BLOCK < k1 ? kk + OR_P_BLOCK : k1, x;
+            double bm = -INFINITY;
             for (x = kk; x < e; ++x)
-                if (s_buf[x - k0] > m_blk) m_blk = s_buf[x - k0];
+                if (s_buf[x - k0] > bm) bm = s_buf[x - k0];
+            if (r == -INFINITY) {
+                r = bm;
+            } else {
+                if (move_is_ambiguous(bm, r)) unverifiable = 1;
+                if (bm * 1.4426950408889634 > r * 1.4426950408889634 + OR_P_LAG_LOG2) r = bm;
+            }
         }
         if (j->pquant) {
-            double y = 256.0 * exp(s - m_blk);
-            pt = or_e4m3_value(or_e4m3_encode(y)) / 256.0 * exp(m_blk - M);
+            double y = OR_P_SCALE * exp(s - r);
+            pt = or_e4m3_value(or_e4m3_encode(y)) / OR_P_SCALE * exp(r - M);
             if (a) {
-                double amb = code_ambiguity(y, s, m_blk) * exp(m_blk - M);
+                double amb = code_ambiguity(y, s, r) * exp(r - M);
                 if (amb > 0.0)
                     for (d = 0; d < j->D; ++d) a[d] += amb * fabs(elem(j, j->v, kk, h, d));
             }
@@ -415,7 +442,8 @@ static void attend_one(const att_job* j, int64_t ri, int h, double* s_buf) {
     }
     for (d = 0; d < j->D; ++d) o[d] = o[d] * dsv / l;
     if (a)
-        for (d = 0; d < j->D; ++d) a[d] = a[d] * dsv / l;
+        for (d = 0; d < j->D; ++d)
+            a[d] = (unverifiable && j->pquant) ? INFINITY : a[d] * dsv / l;
 }
 
 static void* att_worker(void* arg) {

@@ -12,19 +12,24 @@
 //   warp 9       MMA issuer (one lane): S_i = Q_i K^T into TMEM, then
 //                O_i += P_i V (V in shared memory, MN-major)
 //   warps 0-3    softmax for query tile 0, warps 4-7 for tile 1: one thread
-//                per query row (= TMEM lane), running max, exp2 with the
+//                per query row (= TMEM lane), row max, exp2 with the
 //                descales folded into one FMA, row sum of the unquantised
 //                p, P quantised for the PV product, O rescaled in TMEM when
-//                the row max grows, and the bf16 epilogue.
+//                the max that P is taken against changes, and the bf16
+//                epilogue.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512).
 // attn_fwd_kernel (BF16): P_i aliases the first 64 columns of S_i and PV
 // reads it from TMEM; S_i(j+1) is issued after PV_i(j).
 // attn_fwd_fp8_kernel (FP8): P_i goes to shared memory, so S_i(j+1) is
 // computed while the softmax still works on block j (details there).
 //
-// P rule (pages silent; fixed here): p' = 2^(s*c - m + 8) = 256 p with c =
-// ds_q ds_k softmax_scale log2(e) and m the running max of s*c; P = e4m3(p')
-// for the PV product; l accumulates the unquantised p'; out = O ds_v / l.
+// P rule (pages silent; fixed here), per 128-key block: c = ds_q ds_k
+// softmax_scale log2(e), t = s*c; FP8: p' = 2^(t - r + 5) against a reference
+// max r that starts at the first block's max and moves to a later block's
+// max only when that exceeds r by more than 3 (so p' <= 2^8 = 256, never
+// saturating, and O is rescaled only on such moves); BF16: p' = 2^(t - m)
+// with m the running max.  P = e4m3(p') (bf16(p')) for the PV product; l
+// accumulates the unquantised p'; out = O ds_v / l.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -46,6 +51,10 @@ constexpr bool kAlternate = false;
 // Pairs of columns (of every 8) whose exp2 runs on the FMA pipe (polynomial)
 // instead of the MUFU.
 constexpr int kPolyPairsPer8 = 2;
+// FP8 P rule: the reference max moves only past this lag (log2 units), and
+// P = e4m3(2^(t - r + kPOffsetLog2)) stays at or below 2^(kRefLag + kPOffsetLog2) = 256.
+constexpr float kRefLag = 3.0f;
+constexpr float kPOffsetLog2 = 5.0f;
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -711,8 +720,12 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         mx3 = fmax3(mx3, __uint_as_float(u[c + 6]), __uint_as_float(u[c + 7]));
       }
       const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3));
-      const float m_new = fmaxf(m_run, mx * cscale);
-      const float neg = 8.0f - m_new;
+      // reference max: moves to this block's max only when that exceeds it
+      // by more than kRefLag (always on the first block, m_run = -inf)
+      const float m_blk = mx * cscale;
+      const bool moved = m_blk > m_run + kRefLag;
+      const float m_new = moved ? m_blk : m_run;
+      const float neg = kPOffsetLog2 - m_new;
       const uint64_t c2 = f2_pack(cscale, cscale);
       const uint64_t n2 = f2_pack(neg, neg);
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
@@ -749,9 +762,9 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
         sum = a0 + a1;
       }
-      const float alpha = ex2_approx(m_run - m_new);   // 0 on the first block
+      const float alpha = ex2_approx(m_run - m_new);   // 0 on the first block, 1 unless moved
       l_run = l_run * alpha + sum;
-      if (j > 0 && __any_sync(0xFFFFFFFFu, m_new > m_run)) {
+      if (j > 0 && __any_sync(0xFFFFFFFFu, moved)) {
         // O_i holds PV up to block j-1: wait for it before rescaling
         if (!mbar_wait(&bars.pv_done[wg][(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag)) {
           ok = false;

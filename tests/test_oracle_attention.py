@@ -4,8 +4,8 @@ vLLM-Omni docs, "Quantized KV Cache", overview: Q/K/V are quantised
 dynamically right before the (full, non-causal) attention operator.  The
 pages give no numeric attention outputs, so the oracle is pinned by a
 library special case (softmax from scipy with no P quantisation), closed
-forms (Q = 0, a single key, hand-worked two-key cases that exercise the
-e4m3(256 p) rule), and invariants.
+forms (Q = 0, a single key, hand-worked cases that exercise the block rule
+e4m3(32 exp(s - r)) with its lagged reference max r), and invariants.
 """
 import math
 
@@ -98,8 +98,8 @@ def _two_key_case(s1_code):
 
 
 def test_pquant_rule_normal_range():
-    # s = (0, -0.125): p1 = e^-0.125 = 0.88250; 256 p1 = 225.92 lies in
-    # [128, 256) where E4M3 spacing is 16, nearest 224 -> p~1 = 0.875.
+    # s = (0, -0.125): r = 0, p1 = e^-0.125 = 0.88250; 32 p1 = 28.24 lies in
+    # [16, 32) where E4M3 spacing is 2, nearest 28 -> p~1 = 28/32 = 0.875.
     # l is the unquantised sum 1 + e^-0.125.
     q8, k8, v8, cu = _two_key_case(0xA0)      # 0xA0 = -0.125
     o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True)
@@ -115,13 +115,13 @@ def test_pquant_rule_normal_range():
 
 
 def test_pquant_rule_subnormal_range():
-    # s = (0, -12): p1 = e^-12 = 6.144e-6; 256 p1 = 1.573e-3 is below 2^-6,
-    # in the subnormal range with spacing 2^-9 = 1.953e-3, so it rounds to
-    # 2^-9 and p~1 = 2^-9 / 256 = 2^-17.
-    q8, k8, v8, cu = _two_key_case(0xD4)      # 0xD4 = -12.0
+    # s = (0, -8): p1 = e^-8 = 3.3546e-4; 32 p1 = 0.010735 is below 2^-6, in
+    # the subnormal range with spacing 2^-9: 0.010735 / 2^-9 = 5.496 rounds
+    # to 5, so p~1 = 5 * 2^-9 / 32 = 5 * 2^-14.
+    q8, k8, v8, cu = _two_key_case(0xD0)      # 0xD0 = -8.0
     o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True)
-    want = 2.0 ** -17 / (1.0 + math.exp(-12.0))
-    assert abs(o[0, 0, 1] - want) < 1e-20
+    want = 5 * 2.0 ** -14 / (1.0 + math.exp(-8.0))
+    assert abs(o[0, 0, 1] - want) < 1e-18
 
 
 def test_rows_sum_to_one_and_columns_stay_in_range():
@@ -134,8 +134,9 @@ def test_rows_sum_to_one_and_columns_stay_in_range():
     o = oracle.attention_fp8(q8, k8, ones, cu, (0.3, 0.3, 1.0), pquant=False)
     np.testing.assert_allclose(o, 1.0, rtol=0, atol=1e-14)
     oq = oracle.attention_fp8(q8, k8, ones, cu, (0.3, 0.3, 1.0), pquant=True)
-    # |p~ - p| <= p / 16 for normal codes; subnormal p~ adds at most 2^-18 each
-    assert np.all(np.abs(oq - 1.0) <= 2.0 ** -4 + 64 * 2.0 ** -17)
+    # |p~ - p| <= p / 16 for normal codes; a subnormal code is off by at most
+    # half its 2^-9 step, 2^-10 / 32 = 2^-15 per key
+    assert np.all(np.abs(oq - 1.0) <= 2.0 ** -4 + 64 * 2.0 ** -15)
     o = oracle.attention_fp8(q8, k8, v8, cu, (0.3, 0.3, 1.0), pquant=False)
     vv = _decode_torch(v8)
     for b in range(len(lens)):
@@ -154,34 +155,68 @@ def test_row_subset_equals_full_rows():
     np.testing.assert_array_equal(sub, full[rows])
 
 
-def test_pquant_rule_uses_running_block_max():
-    # 129 keys: keys 0..127 score 0 (block 0), key 128 scores 1 (block 1).
-    # Block 0 is quantised against its running max 0: p = 1 -> 256 is exact,
-    # then carried to the final max 1 by the exact factor e^-1, so p~ = e^-1.
-    # (Against the final max it would be e4m3(256 e^-1) = e4m3(94.18) = 96,
-    # p~ = 0.375.)  Key 128: p~ = 1.  l = 128 e^-1 + 1 (unquantised).
+def _block_step_case(s128_code):
+    """129 keys, q = e_0: keys 0..127 score 0 (block 0), key 128 scores
+    value(s128_code) (block 1); v_128 = e_1, v_0 = e_2; one query row."""
     D, n = 128, 129
     q8 = np.zeros((n, 1, D), np.uint8)
     k8 = np.zeros((n, 1, D), np.uint8)
     v8 = np.zeros((n, 1, D), np.uint8)
     q8[:, 0, 0] = 0x38                # q = e_0
-    k8[128, 0, 0] = 0x38              # s_128 = 1
+    k8[128, 0, 0] = s128_code
     v8[128, 0, 1] = 0x38              # v_128 = e_1
     v8[0, 0, 2] = 0x38                # v_0 = e_2
     cu = np.array([0, n], dtype=np.int32)
+    return q8, k8, v8, cu
+
+
+def test_reference_max_stays_when_block_max_is_within_the_lag():
+    # s_128 = 1 < 3 ln 2 = 2.079 (3 in log2 units): r stays 0 (block 0's
+    # max).  Key 128: 32 e^1 = 86.98 lies in [64, 128) with spacing 8 -> 88,
+    # carried to the final max 1: p~ = 88/32 e^-1.  Block 0 keys: 32 e^0 = 32
+    # exact -> p~ = e^-1.  l = 128 e^-1 + 1 (unquantised).
+    q8, k8, v8, cu = _block_step_case(0x38)          # s_128 = 1.0
     o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True,
                              rows=[5])
     l = 128 * math.exp(-1.0) + 1.0
-    assert abs(o[0, 0, 1] - 1.0 / l) < 1e-15
+    assert abs(o[0, 0, 1] - 88.0 / 32.0 * math.exp(-1.0) / l) < 1e-15
     assert abs(o[0, 0, 2] - math.exp(-1.0) / l) < 1e-15
-    assert abs(o[0, 0, 2] - 0.375 / l) > 1e-4       # not the final-max rule
+    # a reference that followed every new max would give key 128 exactly 1
+    assert abs(o[0, 0, 1] - 1.0 / l) > 1e-5
+
+
+def test_reference_max_moves_past_the_lag():
+    # s_128 = 2.5 > 3 ln 2: r moves to 2.5 at block 1, so key 128 gives
+    # 32 e^0 = 32 exactly (p~ = 1); block 0 keys were quantised against r = 0
+    # (32 exactly) and carry e^-2.5.  l = 128 e^-2.5 + 1.
+    q8, k8, v8, cu = _block_step_case(0x42)          # 0x42 = 2.5
+    o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True,
+                             rows=[5])
+    l = 128 * math.exp(-2.5) + 1.0
+    assert abs(o[0, 0, 1] - 1.0 / l) < 1e-15
+    assert abs(o[0, 0, 2] - math.exp(-2.5) / l) < 1e-15
+    # staying at r = 0 would have given e4m3(32 e^2.5) = e4m3(389.8) = 384
+    assert abs(o[0, 0, 1] - 384.0 / 32.0 * math.exp(-2.5) / l) > 1e-5
+
+
+def test_reference_move_at_the_threshold_makes_the_row_unverifiable():
+    # s_128 = 3 ln 2 exactly: the move is decided at the tie, either choice is
+    # a correct result of the rule, so the row's allowance is infinite
+    q8, k8, v8, cu = _block_step_case(0x38)
+    o, amb = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 3.0 * math.log(2.0), 1.0), scale=1.0,
+                                  pquant=True, rows=[5], return_ambiguity=True)
+    assert np.isinf(amb).all()
+    o, amb = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 2.5, 1.0), scale=1.0,
+                                  pquant=True, rows=[5], return_ambiguity=True)
+    assert np.isfinite(amb).all()
 
 
 def test_pquant_block_is_128_keys():
     # keys 0..63 score 0, key 64 scores 1: all in block 0 (128 keys), so
     # keys 0..63 are quantised against the block max 1, giving
-    # e4m3(256 e^-1)/256 = 96/256 = 0.375 (with 64-key blocks they would be
-    # quantised against max 0 and give e^-1 exactly).
+    # e4m3(32 e^-1)/32 = e4m3(11.77)/32 = 12/32 = 0.375 (with 64-key blocks
+    # the reference would be 0, key 64 would stay within the lag, and keys
+    # 0..63 would carry e^-1 exactly).
     D, n = 128, 65
     q8 = np.zeros((n, 1, D), np.uint8)
     k8 = np.zeros((n, 1, D), np.uint8)
@@ -197,8 +232,8 @@ def test_pquant_block_is_128_keys():
 
 
 def test_pquant_block_rule_second_block_lower_max():
-    # block 1's scores are all below block 0's max: its running max is the
-    # same as block 0's, so p~ = e4m3(256 e^s)/256 for s = -0.125 there: 224/256
+    # block 1's scores are all below block 0's max: the reference stays 0, so
+    # p~ = e4m3(32 e^s)/32 for s = -0.125 there: 28/32
     D, n = 128, 130
     q8 = np.zeros((n, 1, D), np.uint8)
     k8 = np.zeros((n, 1, D), np.uint8)
@@ -214,17 +249,17 @@ def test_pquant_block_rule_second_block_lower_max():
 
 
 def test_ambiguity_reported_only_at_rounding_ties():
-    # s1 = ln(232/256): y1 = 256 e^{s1} = 232 is the tie between the E4M3
-    # values 224 and 240, so both codes are correct results of the rule and
-    # the oracle reports the one-step change (16/256) * |v1| / l.
+    # s1 = ln(29/32): y1 = 32 e^{s1} = 29 is the tie between the E4M3 values
+    # 28 and 30, so both codes are correct results of the rule and the oracle
+    # reports the one-step change (2/32) * |v1| / l.
     q8, k8, v8, cu = _two_key_case(0x38)          # k1 = 1.0 * e_0
-    ds_k = math.log(232.0 / 256.0)
+    ds_k = math.log(29.0 / 32.0)
     o, amb = oracle.attention_fp8(q8, k8, v8, cu, (1.0, ds_k, 1.0), scale=1.0, pquant=True,
                                   return_ambiguity=True)
-    l = 1.0 + 232.0 / 256.0
-    assert abs(amb[0, 0, 1] - (16.0 / 256.0) / l) < 1e-12
+    l = 1.0 + 29.0 / 32.0
+    assert abs(amb[0, 0, 1] - (2.0 / 32.0) / l) < 1e-12
     assert amb[0, 0, 0] == 0.0                    # v1 has no component there
-    # y1 = 225.92 (s1 = -0.125) is far from any tie: no allowance
+    # y1 = 28.24 (s1 = -0.125) is far from any tie: no allowance
     q8, k8, v8, cu = _two_key_case(0xA0)
     o, amb = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True,
                                   return_ambiguity=True)
