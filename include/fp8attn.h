@@ -32,9 +32,13 @@
  *     division); A == 0 gives qs = ds = 1.  code = e4m3(fl32(x * qs)).
  *   - Static values are bounds A in activation units with the margin already
  *     applied (the margin multiplies saved values once, at export).
- *   - Attention: s = q8.k8 * ds_q * ds_k * softmax_scale; p = exp(s - m)
- *     with m the running row max; P for the PV product is e4m3(256 p); the
- *     row sum l accumulates the unquantised p; out = bf16(O * ds_v / (256 l)).
+ *   - Attention: s = q8.k8 * ds_q * ds_k * softmax_scale, t = s log2(e);
+ *     per 128-key block, P for the PV product is e4m3(2^(t - r + 5)) with r
+ *     the row's reference max (block 0's max, moved to a later block's max
+ *     only when that exceeds r by more than 3, so P <= 256); the row sum l
+ *     accumulates the unquantised 2^(t - r + 5) carried to a common max;
+ *     out = bf16(O * ds_v / l).  The bf16 entry point takes r = the running
+ *     max and P = bf16(2^(t - r)).
  *
  * Layouts: bf16 sources are addressed as (token, head, channel) with the
  * channel contiguous (head_dim == 128) and element strides `tok_stride`,

@@ -18,7 +18,7 @@
 //                the max that P is taken against changes, and the bf16
 //                epilogue.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512).
-// attn_fwd_kernel (BF16): P_i aliases the first 64 columns of S_i and PV
+// attn_fwd_bf16_kernel: P_i aliases the first 64 columns of S_i and PV
 // reads it from TMEM; S_i(j+1) is issued after PV_i(j).
 // attn_fwd_fp8_kernel (FP8): P_i goes to shared memory, so S_i(j+1) is
 // computed while the softmax still works on block j (details there).
@@ -43,11 +43,6 @@ namespace fp8attn {
 namespace {
 
 constexpr int kThreadsAttn = 320;
-// Softmax scheduling: the two query tiles' softmax warpgroups take turns
-// (tile 0 of key block j, tile 1 of block j, tile 0 of block j+1, ...), so
-// each runs with the SM's exp and FMA pipes to itself while the tensor core
-// works on the other tile's MMAs.
-constexpr bool kAlternate = false;
 // Pairs of columns (of every 8) whose exp2 runs on the FMA pipe (polynomial)
 // instead of the MUFU.
 constexpr int kPolyPairsPer8 = 2;
@@ -59,12 +54,11 @@ constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <bool kFp8>
-struct AttnCfg {
-  static constexpr int kStages = kFp8 ? 4 : 2;
-  static constexpr int kTile = kFp8 ? 16384 : 32768;   // bytes of a 128x128 tile
-  static constexpr int kPCols = kFp8 ? 32 : 64;        // TMEM columns of a P tile
-  static constexpr int kKSteps = kFp8 ? 4 : 8;         // MMAs per 128-deep product
+struct Bf16Cfg {
+  static constexpr int kStages = 2;
+  static constexpr int kTile = 32768;   // bytes of a 128x128 bf16 tile (two 64-column halves)
+  static constexpr int kPCols = 64;     // TMEM columns of a bf16 P tile
+  static constexpr int kKSteps = 8;     // MMAs per 128-deep product
   static constexpr int kSmemTiles = 2 + 2 * kStages;
   static constexpr int kSmemBytes = kSmemTiles * kTile + 1024 /*barriers*/ + 1024 /*align*/;
 };
@@ -81,13 +75,12 @@ struct AttnParams {
 
 struct Barriers {
   uint64_t q_full;
-  uint64_t k_full[4];
-  uint64_t v_full[4];
-  uint64_t kv_empty[4];
+  uint64_t k_full[Bf16Cfg::kStages];
+  uint64_t v_full[Bf16Cfg::kStages];
+  uint64_t kv_empty[Bf16Cfg::kStages];
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_done[2];
-  uint64_t tok[2];        // softmax turn tokens (tile 1 -> tile 0, tile 0 -> tile 1)
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -99,11 +92,10 @@ __device__ __forceinline__ void note_error(AttnParams& p, Bars& bars, uint32_t b
   if (p.err) atomicOr(reinterpret_cast<unsigned int*>(p.err), bit);
 }
 
-template <bool kFp8>
 __global__ void __launch_bounds__(kThreadsAttn, 1)
-attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, AttnParams p) {
-  using C = AttnCfg<kFp8>;
+attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, AttnParams p) {
+  using C = Bf16Cfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -143,7 +135,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_init(&bars.s_full[i], 1);
       mbar_init(&bars.p_full[i], 128);
       mbar_init(&bars.o_done[i], 1);
-      mbar_init(&bars.tok[i], 128);
     }
     mbar_init(&bars.drain, 1);
     bars.abort_flag = 0;
@@ -167,13 +158,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       mbar_expect_tx(&bars.q_full, 2 * C::kTile);
-      for (int i = 0; i < 2; ++i) {
-        if (kFp8) {
-          tma_load_3d(sq + i * C::kTile, &tm_q, &bars.q_full, 0, h, seq0 + q0 + 128 * i);
-        } else {
-          tma_load_3d(sq + i * C::kTile, &tm_q, &bars.q_full, 0, h, seq0 + q0 + 128 * i);
-          tma_load_3d(sq + i * C::kTile + 16384, &tm_q, &bars.q_full, 64, h, seq0 + q0 + 128 * i);
-        }
+      for (int i = 0; i < 2; ++i) {   // two 64-column halves per tile
+        tma_load_3d(sq + i * C::kTile, &tm_q, &bars.q_full, 0, h, seq0 + q0 + 128 * i);
+        tma_load_3d(sq + i * C::kTile + 16384, &tm_q, &bars.q_full, 64, h, seq0 + q0 + 128 * i);
       }
     }
     int issued = 0;
@@ -189,10 +176,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int tok = seq0 + 128 * j;
         mbar_expect_tx(&bars.k_full[st], C::kTile);
         tma_load_3d(sk + st * C::kTile, &tm_k, &bars.k_full[st], 0, h, tok);
-        if (!kFp8) tma_load_3d(sk + st * C::kTile + 16384, &tm_k, &bars.k_full[st], 64, h, tok);
+        tma_load_3d(sk + st * C::kTile + 16384, &tm_k, &bars.k_full[st], 64, h, tok);
         mbar_expect_tx(&bars.v_full[st], C::kTile);
         tma_load_3d(sv + st * C::kTile, &tm_v, &bars.v_full[st], 0, h, tok);
-        if (!kFp8) tma_load_3d(sv + st * C::kTile + 16384, &tm_v, &bars.v_full[st], 64, h, tok);
+        tma_load_3d(sv + st * C::kTile + 16384, &tm_v, &bars.v_full[st], 64, h, tok);
       }
       __syncwarp();
       issued = j + 1;
@@ -207,8 +194,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     const bool leader = lane == 0;
-    const uint32_t id_qk = make_idesc(kFp8 ? 0 : 1, kFp8 ? 0 : 1, 128, 0);
-    const uint32_t id_pv = make_idesc(kFp8 ? 0 : 1, kFp8 ? 0 : 1, 128, 1);
+    const uint32_t id_qk = make_idesc(1, 1, 128, 0);   // bf16 x bf16
+    const uint32_t id_pv = make_idesc(1, 1, 128, 1);
     const uint32_t tS[2] = {tmem + 0, tmem + 128};
     const uint32_t tO[2] = {tmem + 256, tmem + 384};
     // Descriptors are built once; the 14-bit start-address field holds
@@ -231,15 +218,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int kk = 0; kk < C::kKSteps; ++kk) {
         // K-major 128B-swizzled operands: 32 bytes of K per MMA; bf16 tiles
         // hold two 64-column halves 16 KB apart
-        const uint32_t koff = (kFp8 ? 32 * kk : (kk / 4) * 16384 + 32 * (kk % 4)) >> 4;
+        const uint32_t koff = ((kk / 4) * 16384 + 32 * (kk % 4)) >> 4;
         ad[kk] = dq + koff;
         bd[kk] = dk + koff;
       }
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < C::kKSteps; ++kk) {
-          if (kFp8) mma_f8_ss(tS[i], ad[kk], bd[kk], id_qk, kk > 0);
-          else mma_bf16_ss(tS[i], ad[kk], bd[kk], id_qk, kk > 0);
+          mma_bf16_ss(tS[i], ad[kk], bd[kk], id_qk, kk > 0);
         }
         mma_commit(&bars.s_full[i]);
       }
@@ -250,16 +236,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint64_t dv = dv0 + static_cast<uint64_t>(st * kTileStep);
 #pragma unroll
       for (int kk = 0; kk < C::kKSteps; ++kk) {
-        // V is MN-major: K (keys) advances by 32 (fp8) or 16 (bf16) rows of
-        // 128 bytes; the second 64-column half of a bf16 tile sits 16 KB on
-        bd[kk] = dv + ((kFp8 ? 4096 * kk : 2048 * kk) >> 4);
+        // V is MN-major: K (keys) advances by 16 rows of 128 bytes; the
+        // second 64-column half of the tile sits 16 KB on (LBO)
+        bd[kk] = dv + ((2048 * kk) >> 4);
       }
       const uint32_t acc0 = j > 0 ? 1u : 0u;
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < C::kKSteps; ++kk) {
-          if (kFp8) mma_f8_ts(tO[i], tS[i] + 8 * kk, bd[kk], id_pv, kk > 0 ? 1u : acc0);
-          else mma_bf16_ts(tO[i], tS[i] + 8 * kk, bd[kk], id_pv, kk > 0 ? 1u : acc0);
+          mma_bf16_ts(tO[i], tS[i] + 8 * kk, bd[kk], id_pv, kk > 0 ? 1u : acc0);
         }
       }
       __syncwarp();
@@ -312,22 +297,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t lane_off = static_cast<uint32_t>(32 * wq) << 16;
     const uint32_t tS = tmem + 128 * wg + lane_off;
     const uint32_t tO = tmem + 256 + 128 * wg + lane_off;
-    float cscale = p.softmax_scale * kLog2e;
-    float ds_v = 1.0f;
-    if (kFp8) {
-      cscale = __ldg(p.descale + 0) * __ldg(p.descale + 1) * cscale;
-      ds_v = __ldg(p.descale + 2);
-    }
-    const float p_off = kFp8 ? 8.0f : 0.0f;   // 2^8 = 256: P scale for E4M3
+    const float cscale = p.softmax_scale * kLog2e;
+    const float ds_v = 1.0f;
+    const float p_off = 0.0f;   // bf16 P = 2^(t - m), no scale needed
     float m_run = -INFINITY;
     float l_run = 0.0f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      if (kAlternate) {
-        // wait for the other warpgroup's turn to end
-        if (wg == 0 && j > 0 && !mbar_wait(&bars.tok[0], (j - 1) & 1, abort_flag)) { ok = false; break; }
-        if (wg == 1 && !mbar_wait(&bars.tok[1], j & 1, abort_flag)) { ok = false; break; }
-      }
       if (!mbar_wait(&bars.s_full[wg], j & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       uint32_t u[128];
@@ -375,13 +351,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         acc[k & 3] = f2_add(acc[k & 3], e);
         float e0, e1;
         f2_unpack(e, e0, e1);
-        if (kFp8) {
-          const uint32_t h = cvt_e4m3x2(e0, e1);
-          if (k & 1) pw[k >> 1] |= h << 16;
-          else pw[k >> 1] = h;
-        } else {
-          pw[k] = cvt_bf16x2(e0, e1);
-        }
+        pw[k] = cvt_bf16x2(e0, e1);
       }
       float sum;
       {
@@ -394,7 +364,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const float alpha = ex2_approx(m_run - m_new);   // 0 on the first tile
       l_run = l_run * alpha + sum;
       tmem_st32(tS + 0, *reinterpret_cast<const uint32_t(*)[32]>(&pw[0]));
-      if (!kFp8) tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pw[32]));
+      tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pw[32]));
       // O_i is stable here (PV_i(j-1) finished before S_i(j) was written)
       if (j > 0 && __any_sync(0xFFFFFFFFu, m_new > m_run)) {
         const uint64_t a2 = f2_pack(alpha, alpha);
@@ -419,10 +389,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bars.p_full[wg]);
-      if (kAlternate) {
-        if (wg == 0) mbar_arrive(&bars.tok[1]);
-        else if (j + 1 < nkv) mbar_arrive(&bars.tok[0]);
-      }
     }
     if (!ok) {
       if (lane == 0) note_error(p, bars, kErrTimeout);
@@ -869,14 +835,13 @@ bool make_qkv_map(CUtensorMap* m, const void* base, int64_t T, int H, bool bf16)
 
 template <bool kFp8>
 cudaError_t launch_attention_t(const AttnLaunch& a, int64_t T, cudaStream_t stream) {
-  using C = AttnCfg<kFp8>;
   CUtensorMap mq, mk, mv;
   if (!make_qkv_map(&mq, a.q, T, a.heads, !kFp8) || !make_qkv_map(&mk, a.k, T, a.heads, !kFp8) ||
       !make_qkv_map(&mv, a.v, T, a.heads, !kFp8))
     return cudaErrorInvalidValue;
   // FP8 runs the P-in-shared-memory kernel; BF16 keeps P in TMEM
-  auto kernel = kFp8 ? attn_fwd_fp8_kernel : attn_fwd_kernel<false>;
-  const int smem_bytes = kFp8 ? Fp8Cfg::kSmemBytes : C::kSmemBytes;
+  auto kernel = kFp8 ? attn_fwd_fp8_kernel : attn_fwd_bf16_kernel;
+  const int smem_bytes = kFp8 ? Fp8Cfg::kSmemBytes : Bf16Cfg::kSmemBytes;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

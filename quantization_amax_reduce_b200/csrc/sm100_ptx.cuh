@@ -77,21 +77,6 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// try_wait that lets the hardware suspend the thread until the phase
-// completes or `suspend_ns` elapses, so waiting warps take no issue slots.
-__device__ __forceinline__ bool mbar_test_suspend(uint64_t* bar, uint32_t parity,
-                                                  uint32_t suspend_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.b32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
-      : "memory");
-  return ok != 0;
-}
-
 // Wait until the phase with the given parity has completed.  Returns false
 // if the wait ran past kWaitLimitNs or `abort_flag` (shared memory, may be
 // null) became non-zero.  Spins on try_wait (no suspend hint: a suspended
@@ -179,17 +164,6 @@ __device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
-// D(tmem) (+)= A(tmem) * B(smem desc), E4M3 x E4M3 -> F32
-__device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                          uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // BF16 x BF16 -> F32, operands from shared memory.
 __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                             uint32_t idesc, uint32_t accumulate) {
@@ -267,15 +241,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
-// Load 16 consecutive columns of this thread's lane.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-      : FP8ATTN_R8(0), FP8ATTN_R8(8)
-      : "r"(taddr));
-}
-
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -288,24 +253,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
           taddr),
       FP8ATTN_W8(0), FP8ATTN_W8(8), FP8ATTN_W8(16), FP8ATTN_W8(24)
-      : "memory");
-}
-
-// Store 16 consecutive columns of this thread's lane.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-      FP8ATTN_W8(0), FP8ATTN_W8(8)
-      : "memory");
-}
-
-// Store 8 consecutive columns of this thread's lane.
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
-      FP8ATTN_W8(0)
       : "memory");
 }
 
