@@ -227,6 +227,16 @@ fp8attn_status fp8attn_parse_selector(const char* text, int max_index, uint8_t* 
  * -1 on a bad argument. */
 int fp8attn_select_mode(const fp8attn_ctx* ctx, const uint8_t* skip_mask, int layer);
 
+/* Mode of one attention call inside a denoising loop (vLLM-Omni docs,
+ * parameters table: kv_cache_skip_steps and kv_cache_skip_layers; listed
+ * steps or layers skip FP8 attention): SKIP if skip_steps[step] or
+ * skip_layers[layer], else as fp8attn_select_mode.  Either mask may be NULL;
+ * skip_steps holds num_steps entries (a fp8attn_parse_selector mask).  -1 on
+ * a bad argument (layer out of range, or step outside [0, num_steps) when
+ * skip_steps is given). */
+int fp8attn_select_mode_at_step(const fp8attn_ctx* ctx, const uint8_t* skip_layers, int layer,
+                                const uint8_t* skip_steps, int num_steps, int step);
+
 /* E4M3 cast helper: d_out[i] = e4m3(fl32(d_in[i] * scale)), fp32 device
  * input, n elements, the same conversion the quantisation kernel uses. */
 fp8attn_status fp8attn_e4m3_encode(const float* d_in, int64_t n, float scale, void* d_out,

@@ -311,3 +311,13 @@ def layer_mode(layer: int, skip: Iterable[int], has_static: bool) -> int:
     if layer in set(skip):
         return SKIP
     return STATIC if has_static else DYNAMIC
+
+
+def step_layer_mode(layer: int, step: int, skip_layers: Iterable[int], skip_steps: Iterable[int],
+                    has_static: bool) -> int:
+    """vLLM-Omni parameters table (kv_cache_skip_steps, kv_cache_skip_layers):
+    listed denoising steps or layers keep the native dtype (SKIP); every other
+    call uses the FP8 path, STATIC once static scales are set, else DYNAMIC."""
+    if step in set(skip_steps):
+        return SKIP
+    return layer_mode(layer, skip_layers, has_static)

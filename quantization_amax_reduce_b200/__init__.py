@@ -89,6 +89,7 @@ def lib() -> ctypes.CDLL:
         "fp8attn_read_error_word": (I, [P, P]),
         "fp8attn_parse_selector": (I, [ctypes.c_char_p, I, U8P]),
         "fp8attn_select_mode": (I, [P, U8P, I]),
+        "fp8attn_select_mode_at_step": (I, [P, U8P, I, U8P, I, I]),
         "fp8attn_e4m3_encode": (I, [P, I64, F, P, P]),
         "fp8attn_launch_count": (ctypes.c_uint64, []),
         "fp8attn_quantize_qkv_noalloc": (I, [P, P, P, I64, I64, P, P, I, I, I64, I, I, P, P, P, P,
@@ -286,6 +287,20 @@ class Context:
                                       layer)
         if r < 0:
             raise FP8AttnError(1, "fp8attn_select_mode")
+        return r
+
+    def select_mode_at_step(self, layer: int, step: int, skip_layers: Optional[np.ndarray] = None,
+                            skip_steps: Optional[np.ndarray] = None) -> int:
+        """Mode of layer `layer` at denoising step `step`: SKIP if either mask
+        selects it, else STATIC/DYNAMIC as select_mode."""
+        ml = None if skip_layers is None else np.ascontiguousarray(skip_layers, dtype=np.uint8)
+        ms = None if skip_steps is None else np.ascontiguousarray(skip_steps, dtype=np.uint8)
+        r = lib().fp8attn_select_mode_at_step(
+            self._h, None if ml is None else ml.ctypes.data_as(ctypes.c_void_p), layer,
+            None if ms is None else ms.ctypes.data_as(ctypes.c_void_p),
+            0 if ms is None else int(ms.size), step)
+        if r < 0:
+            raise FP8AttnError(1, "fp8attn_select_mode_at_step")
         return r
 
 

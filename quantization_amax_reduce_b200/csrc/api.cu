@@ -427,6 +427,14 @@ int fp8attn_select_mode(const fp8attn_ctx* ctx, const uint8_t* skip_mask, int la
   return ctx->has_static[layer] ? FP8ATTN_STATIC : FP8ATTN_DYNAMIC;
 }
 
+int fp8attn_select_mode_at_step(const fp8attn_ctx* ctx, const uint8_t* skip_layers, int layer,
+                                const uint8_t* skip_steps, int num_steps, int step) {
+  if (!layer_ok(ctx, layer)) return -1;
+  if (skip_steps && (step < 0 || step >= num_steps)) return -1;
+  if (skip_steps && skip_steps[step]) return FP8ATTN_SKIP;
+  return fp8attn_select_mode(ctx, skip_layers, layer);
+}
+
 fp8attn_status fp8attn_e4m3_encode(const float* d_in, int64_t n, float scale, void* d_out,
                                    void* stream) {
   if (n < 0 || (n > 0 && (!d_in || !d_out))) return FP8ATTN_ERR_INVALID;

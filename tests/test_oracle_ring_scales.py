@@ -124,3 +124,17 @@ def test_layer_modes():
     assert oracle.layer_mode(3, skip, False) == oracle.DYNAMIC
     assert oracle.layer_mode(3, skip, True) == oracle.STATIC
     assert oracle.layer_mode(2, skip, True) == oracle.SKIP
+
+
+def test_step_and_layer_modes_follow_both_selectors():
+    # vLLM-Omni parameters table: listed steps or layers skip FP8 attention;
+    # the table's own examples, "0,1,4-6" for steps and "0-2,10" for layers
+    steps = oracle.parse_selector("0,1,4-6", 50)
+    layers = oracle.parse_selector("0-2,10", 24)
+    for step in range(50):
+        for layer in range(24):
+            want_skip = step in (0, 1, 4, 5, 6) or layer in (0, 1, 2, 10)
+            m = oracle.step_layer_mode(layer, step, layers, steps, False)
+            assert m == (oracle.SKIP if want_skip else oracle.DYNAMIC), (step, layer)
+            m = oracle.step_layer_mode(layer, step, layers, steps, True)
+            assert m == (oracle.SKIP if want_skip else oracle.STATIC), (step, layer)
