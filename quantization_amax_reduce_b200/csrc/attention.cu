@@ -34,6 +34,9 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
+#include <cstdint>
+#include <mutex>
+
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 #include "state.cuh"
@@ -44,8 +47,11 @@ namespace {
 
 constexpr int kThreadsAttn = 320;
 // Pairs of columns (of every 8) whose exp2 runs on the FMA pipe (polynomial)
-// instead of the MUFU.
+// instead of the MUFU, BF16 kernel (the last two of each eight).
 constexpr int kPolyPairsPer8 = 2;
+// FP8 kernel: every kPolyEvery-th column pair takes the polynomial (the same
+// 25 %, spread evenly through the loop: measured 1 % faster there).
+constexpr int kPolyEvery = 4;
 // FP8 P rule: the reference max moves only past this lag (log2 units), and
 // P = e4m3(2^(t - r + kPOffsetLog2)) stays at or below 2^(kRefLag + kPOffsetLog2) = 256.
 constexpr float kRefLag = 3.0f;
@@ -703,7 +709,7 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         float t0, t1;
         f2_unpack(t, t0, t1);
         uint64_t e;
-        if ((k & 7) >= 8 - kPolyPairsPer8)
+        if (k % kPolyEvery == kPolyEvery - 1)
           e = f2_exp2_poly(f2_pack(fmaxf(t0, -126.0f), fmaxf(t1, -126.0f)));
         else
           e = f2_pack(ex2_approx(t0), ex2_approx(t1));
@@ -842,12 +848,21 @@ cudaError_t launch_attention_t(const AttnLaunch& a, int64_t T, cudaStream_t stre
   // FP8 runs the P-in-shared-memory kernel; BF16 keeps P in TMEM
   auto kernel = kFp8 ? attn_fwd_fp8_kernel : attn_fwd_bf16_kernel;
   const int smem_bytes = kFp8 ? Fp8Cfg::kSmemBytes : Bf16Cfg::kSmemBytes;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         smem_bytes);
+  // the shared-memory opt-in is a per-device function attribute: set it once
+  // for each device this process launches on
+  static std::mutex mu;
+  static uint64_t attr_set = 0;   // bit d: done on device d
+  {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!(attr_set >> dev & 1u)) {
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+      if (e != cudaSuccess) return e;
+      attr_set |= uint64_t{1} << dev;
+    }
   }
   AttnParams p;
   p.cu = a.cu;
