@@ -60,7 +60,7 @@ def test_bf16_attention_small_shapes(lens, H):
 
 
 def test_sharp_softmax_rescales():
-    """Large score range so the running max moves across key tiles (O
+    """Large score range so the reference max moves across key tiles (O
     rescaling in TMEM) and many p fall in E4M3's subnormal range."""
     lens = [900]
     H = 2
@@ -145,3 +145,28 @@ def test_bad_cu_seqlens_sets_error_word():
     assert (out[100:] == 7.0).all()       # the broken sequence wrote nothing
     assert (out[:100] == 0.0).all()       # the valid one attends to zeros
     assert qar.read_error_word(err) == 0
+
+
+def test_reference_max_stays_and_moves_by_design():
+    """Block maxima chosen so the reference max stays within the lag (block 1:
+    +1.5 = +2.16 in log2 units), moves past it (block 2: +3.0 over the
+    reference = +4.33), stays again (block 3), and sees a lower block (4);
+    the other keys score below 0.6.  Exercised for rows of both query tiles."""
+    n, H, D = 5 * 128, 1, 128
+    cu = np.array([0, n], dtype=np.int32)
+    g = torch.Generator().manual_seed(21)
+    q = torch.zeros(n, H, D)
+    q[:, :, 0] = 1.0
+    k = torch.zeros(n, H, D)
+    k[:, :, 0] = torch.rand(n, H, generator=g) * 0.6          # background scores
+    for blk, x in enumerate((1.0, 2.5, 4.0, 5.5, 3.0)):       # one maximum per block
+        k[128 * blk + 17, :, 0] = x
+    v = torch.randn(n, H, D, generator=g) * 0.5
+    q8, k8, v8 = (t.to(torch.float8_e4m3fn).view(torch.uint8) for t in (q, k, v))
+    ds = [1.0, 1.0, 1.0]
+    out = qar.varlen_fwd(q8.to(DEV), k8.to(DEV), v8.to(DEV), torch.as_tensor(cu, device=DEV), n,
+                         torch.tensor(ds, device=DEV), softmax_scale=1.0)
+    want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds, scale=1.0,
+                                return_ambiguity=True)
+    assert np.isfinite(want[1]).all()                         # no decision at a tie
+    assert_attention_close(out, want, what="reference max stays and moves")
