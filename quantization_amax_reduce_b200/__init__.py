@@ -349,7 +349,8 @@ def varlen_fwd_bf16(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlen
                     max_seqlen: int, softmax_scale: float = 0.0,
                     out: Optional[torch.Tensor] = None, error: Optional[torch.Tensor] = None,
                     stream=None) -> torch.Tensor:
-    """Native bf16 attention for skipped layers (same kernel, bf16 MMAs)."""
+    """Native bf16 attention for skipped layers or steps (bf16 MMAs, P kept in
+    TMEM, running row max, no quantisation)."""
     T, H, cu, out = _attn_common(q, k, v, cu_seqlens, out, torch.bfloat16)
     _check(lib().fp8attn_varlen_fwd_bf16(_ptr(q), _ptr(k), _ptr(v), _ptr(cu), cu.numel() - 1,
                                          int(max_seqlen), T, H, HEAD_DIM, float(softmax_scale),
