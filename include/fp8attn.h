@@ -242,6 +242,19 @@ int fp8attn_select_mode_at_step(const fp8attn_ctx* ctx, const uint8_t* skip_laye
 fp8attn_status fp8attn_e4m3_encode(const float* d_in, int64_t n, float scale, void* d_out,
                                    void* stream);
 
+/* Self-test of the bounded waits (failure detection without a GPU fault).
+ * The pages have no counterpart: every wait inside this library's kernels
+ * (mbarrier waits of the attention kernels, the grid barrier of the
+ * quantisation kernels) gives up after a time limit and reports
+ * FP8ATTN_ERR_TIMEOUT instead of hanging.  This runs two probes on `stream`
+ * whose waits nothing ever completes -- an mbarrier wait with limit
+ * `mbar_limit_ns` (0 < limit <= 1 s) and a two-CTA grid barrier that one CTA
+ * leaves before arriving (limit 1 s) -- synchronises the stream, and stores
+ * in *h_gave_up how many of the two waits gave up (2 when the bounds work).
+ * Returns FP8ATTN_ERR_INVALID for a bad limit or null output,
+ * FP8ATTN_ERR_CUDA on a CUDA error.  Takes about 1 s. */
+int fp8attn_selftest_bounded_waits(uint64_t mbar_limit_ns, int* h_gave_up, void* stream);
+
 /* Allocation-free one-shot dynamic quantisation.  The pages have no
  * counterpart to this entry point; it exists for callers that cannot
  * allocate device memory -- for example an operator that an inference

@@ -95,6 +95,7 @@ def lib() -> ctypes.CDLL:
         "fp8attn_quantize_qkv_noalloc": (I, [P, P, P, I64, I64, P, P, I, I, I64, I, I, P, P, P, P,
                                              P, P]),
         "fp8attn_quantize_qkv_noalloc_error": (I, [P]),
+        "fp8attn_selftest_bounded_waits": (I, [ctypes.c_uint64, ctypes.POINTER(I), P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -474,3 +475,15 @@ def save_scale_file(path: str, layer_names: Sequence[str], values: np.ndarray) -
             for n, v in zip(layer_names, values)}
     with open(path, "w") as f:
         json.dump(data, f, indent=2)
+
+
+def selftest_bounded_waits(mbar_limit_ns: int = 50_000_000, device=None) -> int:
+    """Run the library's two wait probes (an mbarrier wait and a grid barrier
+    that nothing completes) and return how many gave up at their limit (2 when
+    the bounds work).  Takes about one second."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    n = ctypes.c_int(-1)
+    _check(lib().fp8attn_selftest_bounded_waits(int(mbar_limit_ns), ctypes.byref(n),
+                                                ctypes.c_void_p(_stream(None, dev))),
+           "fp8attn_selftest_bounded_waits")
+    return n.value

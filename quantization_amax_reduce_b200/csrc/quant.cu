@@ -529,7 +529,67 @@ cudaError_t noalloc_scratch(uint32_t** out) {
 
 }  // namespace fp8attn
 
+// ---------------------------------------------------------------------------
+// Self-test of the bounded waits: failure detection without a GPU fault.
+// Each probe waits on something that never completes; the wait must give up
+// at its limit and report it, and the GPU stays usable.
+// ---------------------------------------------------------------------------
+namespace fp8attn {
+namespace {
+
+__device__ GlobalState g_probe_state;     // grid-barrier words used only here
+__device__ int32_t g_probe_result[2];     // per probe: 1 = the wait completed, 2 = gave up
+
+// An mbarrier that nothing arrives on: mbar_wait_limit (the wait of the
+// attention kernels, with a caller-chosen limit) must give up.
+__global__ void mbar_timeout_probe(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const bool done = mbar_wait_limit(&bar, 0, nullptr, limit_ns);
+  if (threadIdx.x == 0) g_probe_result[0] = done ? 1 : 2;
+}
+
+// The quantisation kernels' grid barrier with one of two CTAs leaving before
+// it arrives: the other must give up after kWaitLimitNs.
+__global__ void grid_barrier_timeout_probe() {
+  __shared__ int s_ok;
+  if (blockIdx.x == 1) return;
+  const bool ok = grid_barrier(&g_probe_state, &s_ok);
+  if (threadIdx.x == 0) g_probe_result[1] = ok ? 1 : 2;
+}
+
+}  // namespace
+}  // namespace fp8attn
+
 extern "C" {
+
+// See include/fp8attn.h.
+int fp8attn_selftest_bounded_waits(uint64_t mbar_limit_ns, int* h_gave_up, void* stream) {
+  using namespace fp8attn;
+  if (!h_gave_up || mbar_limit_ns == 0 || mbar_limit_ns > kWaitLimitNs) return 1;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const GlobalState zero_state{};
+  const int32_t zero_result[2] = {0, 0};
+  if (cudaMemcpyToSymbolAsync(g_probe_state, &zero_state, sizeof(zero_state), 0,
+                              cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyToSymbolAsync(g_probe_result, zero_result, sizeof(zero_result), 0,
+                              cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return 2;
+  mbar_timeout_probe<<<1, 32, 0, s>>>(mbar_limit_ns);
+  grid_barrier_timeout_probe<<<2, 32, 0, s>>>();
+  if (cudaGetLastError() != cudaSuccess) return 2;
+  int32_t result[2] = {0, 0};
+  if (cudaMemcpyFromSymbolAsync(result, g_probe_result, sizeof(result), 0,
+                                cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return 2;
+  *h_gave_up = (result[0] == 2 ? 1 : 0) + (result[1] == 2 ? 1 : 0);
+  return 0;
+}
 
 // See include/fp8attn.h.
 int fp8attn_quantize_qkv_noalloc(const void* q, const void* k, const void* v, int64_t tok_stride,

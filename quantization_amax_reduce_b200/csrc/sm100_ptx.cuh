@@ -78,21 +78,28 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed.  Returns false
-// if the wait ran past kWaitLimitNs or `abort_flag` (shared memory, may be
+// if the wait ran past `limit_ns` or `abort_flag` (shared memory, may be
 // null) became non-zero.  Spins on try_wait (no suspend hint: a suspended
 // thread can wake well after the phase completes); the limit and the abort
 // flag are checked every 64 tries.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          const volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity,
+                                                const volatile int* abort_flag,
+                                                uint64_t limit_ns) {
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_test(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (abort_flag && *abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+      if (global_timer_ns() - t0 > limit_ns) return false;
     }
   }
+}
+
+// The wait every kernel of this library uses: bounded by kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          const volatile int* abort_flag) {
+  return mbar_wait_limit(bar, parity, abort_flag, kWaitLimitNs);
 }
 
 // ---------------------------------------------------------------------------

@@ -94,6 +94,11 @@ def test_host_argument_checks_need_no_gpu(L):
                                 None, None) == 0
     assert L.fp8attn_create(0, P(256), 1 << 20, None, ctypes.byref(P())) == 1
     assert L.fp8attn_e4m3_encode(None, 5, 1.0, None, None) == 1
+    # the wait self-test checks its limit (0 < limit <= 1 s) and output first
+    n = ctypes.c_int(0)
+    assert L.fp8attn_selftest_bounded_waits(ctypes.c_uint64(0), ctypes.byref(n), None) == 1
+    assert L.fp8attn_selftest_bounded_waits(ctypes.c_uint64(2 * 10**9), ctypes.byref(n), None) == 1
+    assert L.fp8attn_selftest_bounded_waits(ctypes.c_uint64(10**6), None, None) == 1
 
 
 def test_scale_file_round_trip(tmp_path, golden_dir):
