@@ -82,7 +82,10 @@ typedef enum {
 typedef enum {
   FP8ATTN_DYNAMIC = 0, /* amax ring, current pass included */
   FP8ATTN_STATIC = 1,  /* static bounds set by fp8attn_set_static_scales */
-  FP8ATTN_SKIP = 2     /* native bf16 attention, no quantisation */
+  FP8ATTN_SKIP = 2,    /* native bf16 attention, no quantisation */
+  FP8ATTN_RING = 3     /* cast with the layer's current ring scales (the last ring
+                          update), no amax pass, ring unchanged: the cast step of a
+                          head-sharded dynamic pass (fp8attn_amax_qkv) */
 } fp8attn_mode;
 
 typedef struct fp8attn_ctx fp8attn_ctx;
@@ -113,7 +116,8 @@ fp8attn_status fp8attn_destroy(fp8attn_ctx* ctx);
  * launches plus unpadding).
  *   mode DYNAMIC: amax of each tensor over its valid tokens; push into the
  *     layer's ring; A = ring max; cast with qs = 448/A.  STATIC: cast with the
- *     layer's static bounds (error INVALID if none were set).  SKIP: INVALID.
+ *     layer's static bounds (error INVALID if none were set).  RING: cast with
+ *     the layer's current scales, ring unchanged.  SKIP: INVALID.
  *   q, k, v: bf16 sources; element (t_src, h, d) at base + t_src*tok_stride
  *     + h*head_stride + d.  d_src_seq_start: NULL if the source is packed
  *     (t_src = t); else int32[batch], the source row of each sequence's first
@@ -129,6 +133,22 @@ fp8attn_status fp8attn_quantize_qkv(fp8attn_ctx* ctx, int layer, int mode, const
                                     const int32_t* d_cu_seqlens, int batch, int max_seqlen,
                                     int64_t total_tokens, int num_heads, int head_dim, void* q8,
                                     void* k8, void* v8, void* stream);
+
+/* Per-tensor amax of Q, K and V over their valid tokens into d_amax3 (device
+ * float[3]; NaN ignored, an infinite amax stays infinite), without casting
+ * and without touching any ring (vLLM FP8 ViT page, usage section: the ring
+ * holds observed Q/K/V amax values).  With heads sharded across GPUs, each
+ * rank runs this on its shard, the three values are all-reduced with MAX,
+ * pushed with fp8attn_amax_ring_update, and each shard is cast with mode
+ * FP8ATTN_RING: codes, scales and ring then equal those of one DYNAMIC pass
+ * over all heads.  Sources and errors as fp8attn_quantize_qkv (no outputs);
+ * uses the context's reduction words, so it must not overlap another call
+ * on the same context. */
+fp8attn_status fp8attn_amax_qkv(fp8attn_ctx* ctx, const void* q, const void* k, const void* v,
+                                int64_t tok_stride, int64_t head_stride,
+                                const int32_t* d_src_seq_start, const int32_t* d_cu_seqlens,
+                                int batch, int max_seqlen, int64_t total_tokens, int num_heads,
+                                int head_dim, float* d_amax3, void* stream);
 
 /* Push three externally observed amax values (device float[3]: q, k, v) into
  * the layer's rings and recompute its scales, on the device (vLLM FP8 ViT

@@ -33,7 +33,7 @@ __all__ = [
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libfp8attn.so")
 
-DYNAMIC, STATIC, SKIP = 0, 1, 2
+DYNAMIC, STATIC, SKIP, RING = 0, 1, 2, 3
 RING_LENGTH = 16
 DEFAULT_MARGIN = 1.5
 HEAD_DIM = 128
@@ -74,6 +74,7 @@ def lib() -> ctypes.CDLL:
         "fp8attn_quantize_qkv": (I, [P, I, I, P, P, P, I64, I64, P, P, I, I, I64, I, I, P, P, P,
                                      P]),
         "fp8attn_amax_ring_update": (I, [P, I, P, P]),
+        "fp8attn_amax_qkv": (I, [P, P, P, P, I64, I64, P, P, I, I, I64, I, I, P, P]),
         "fp8attn_set_static_scales": (I, [P, I, F, F, F, P]),
         "fp8attn_clear_static_scales": (I, [P, I]),
         "fp8attn_has_static_scales": (I, [P, I]),
@@ -121,6 +122,32 @@ def _stream(stream, device) -> int:
     if isinstance(stream, torch.cuda.Stream):
         return stream.cuda_stream
     return int(stream)
+
+
+def _qkv_source(q, k, v, cu_seqlens, total_tokens, src_seq_start):
+    """Checks shared by the quantisation entry points; returns (H, tok_stride,
+    head_stride, cu, B, total_tokens, src_seq_start tensor or None)."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _require_cuda(t, name)
+        if t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} must be bfloat16")
+    if q.shape != k.shape or q.shape != v.shape or q.stride() != k.stride() or \
+            q.stride() != v.stride():
+        raise ValueError("q, k, v must share shape and strides")
+    if q.shape[-1] != HEAD_DIM or q.stride(-1) != 1:
+        raise ValueError("head_dim must be 128 and contiguous")
+    H = q.shape[-2]
+    head_stride, tok_stride = q.stride(-2), q.stride(-3)
+    cu = _cu_tensor(cu_seqlens, q.device)
+    B = cu.numel() - 1
+    if total_tokens is None:
+        if src_seq_start is not None:
+            raise ValueError("total_tokens is required with a padded source")
+        total_tokens = q.shape[-3] if q.dim() == 3 else q.shape[0] * q.shape[1]
+    sss = None
+    if src_seq_start is not None:
+        sss = _cu_tensor(src_seq_start, q.device)
+    return H, tok_stride, head_stride, cu, B, total_tokens, sss
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -177,27 +204,10 @@ class Context:
         Q, K, V.  Sources are bf16 with the channel contiguous: packed
         [T, H, 128], padded [B, S_max, H, 128] (pass ``src_seq_start``), or any
         strided view (e.g. slices of a fused [T, 3, H, 128] projection).
-        Returns packed uint8 E4M3 codes [T, H, 128]."""
-        for name, t in (("q", q), ("k", k), ("v", v)):
-            _require_cuda(t, name)
-            if t.dtype != torch.bfloat16:
-                raise ValueError(f"{name} must be bfloat16")
-        if q.shape != k.shape or q.shape != v.shape or q.stride() != k.stride() or \
-                q.stride() != v.stride():
-            raise ValueError("q, k, v must share shape and strides")
-        if q.shape[-1] != HEAD_DIM or q.stride(-1) != 1:
-            raise ValueError("head_dim must be 128 and contiguous")
-        H = q.shape[-2]
-        head_stride, tok_stride = q.stride(-2), q.stride(-3)
-        cu = _cu_tensor(cu_seqlens, q.device)
-        B = cu.numel() - 1
-        if total_tokens is None:
-            if src_seq_start is not None:
-                raise ValueError("total_tokens is required with a padded source")
-            total_tokens = q.shape[-3] if q.dim() == 3 else q.shape[0] * q.shape[1]
-        sss = None
-        if src_seq_start is not None:
-            sss = _cu_tensor(src_seq_start, q.device)
+        Returns packed uint8 E4M3 codes [T, H, 128].  Mode RING casts with the
+        layer's current ring scales (the cast step of a head-sharded pass)."""
+        H, tok_stride, head_stride, cu, B, total_tokens, sss = _qkv_source(
+            q, k, v, cu_seqlens, total_tokens, src_seq_start)
         if out is None:
             out = [torch.empty((total_tokens, H, HEAD_DIM), dtype=torch.uint8, device=q.device)
                    for _ in range(3)]
@@ -207,6 +217,22 @@ class Context:
             _ptr(out[1]), _ptr(out[2]), ctypes.c_void_p(_stream(stream, q.device))),
             "fp8attn_quantize_qkv")
         return out[0], out[1], out[2]
+
+    def amax_qkv(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens,
+                 max_seqlen: int, *, total_tokens: Optional[int] = None, src_seq_start=None,
+                 out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """Per-tensor amax (q, k, v) over the valid tokens into a device fp32
+        [3] tensor; nothing is cast and no ring changes (sources as
+        quantize_qkv)."""
+        H, tok_stride, head_stride, cu, B, total_tokens, sss = _qkv_source(
+            q, k, v, cu_seqlens, total_tokens, src_seq_start)
+        if out is None:
+            out = torch.empty(3, dtype=torch.float32, device=q.device)
+        _check(lib().fp8attn_amax_qkv(
+            self._h, _ptr(q), _ptr(k), _ptr(v), tok_stride, head_stride, _ptr(sss), _ptr(cu), B,
+            int(max_seqlen), int(total_tokens), H, HEAD_DIM, _ptr(out),
+            ctypes.c_void_p(_stream(stream, q.device))), "fp8attn_amax_qkv")
+        return out
 
     def amax_ring_update(self, layer: int, amax3: torch.Tensor, stream=None) -> None:
         """Push three device-side fp32 amax values (q, k, v) into the rings."""
@@ -487,3 +513,24 @@ def selftest_bounded_waits(mbar_limit_ns: int = 50_000_000, device=None) -> int:
                                                 ctypes.c_void_p(_stream(None, dev))),
            "fp8attn_selftest_bounded_waits")
     return n.value
+
+
+def head_sharded_dynamic_quantize(ctx: "Context", layer: int, q: torch.Tensor, k: torch.Tensor,
+                                  v: torch.Tensor, cu_seqlens, max_seqlen: int, group=None,
+                                  out: Optional[Sequence[torch.Tensor]] = None, stream=None
+                                  ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """One dynamic pass over this rank's heads of a layer whose heads are
+    sharded across the ranks of `group` (torch.distributed, NCCL on GPUs):
+    local amax -> all-reduce MAX of the three values (the only exchange) ->
+    push into this rank's ring -> cast this shard with the ring scales.  Every
+    rank ends with the ring, scales and codes one DYNAMIC pass over all heads
+    would give.  With no process group (or one rank) it is the same sequence
+    without the all-reduce."""
+    import torch.distributed as dist
+    amax = ctx.amax_qkv(q, k, v, cu_seqlens, max_seqlen, stream=stream)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+        s = torch.cuda.current_stream(q.device) if stream is None else stream
+        with torch.cuda.stream(s if isinstance(s, torch.cuda.Stream) else torch.cuda.ExternalStream(int(s))):
+            dist.all_reduce(amax, op=dist.ReduceOp.MAX, group=group)
+    ctx.amax_ring_update(layer, amax, stream=stream)
+    return ctx.quantize_qkv(layer, RING, q, k, v, cu_seqlens, max_seqlen, out=out, stream=stream)

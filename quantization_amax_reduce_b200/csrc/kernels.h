@@ -15,9 +15,17 @@ struct QuantLaunch {
   const int32_t* src_seq_start;  // device [batch] or null
   int batch, heads, max_seqlen;
   int64_t total_tokens;          // must equal cu[batch]
-  int dynamic;                   // 1 = ring mode, 0 = static bounds
+  int kind;                      // a QuantKind
+  float* amax_out;               // kQuantAmaxOnly: device float[3]
   void* gs;                      // GlobalState*
   void* ls;                      // LayerState*
+};
+
+enum QuantKind {
+  kQuantStatic = 0,     // cast with the static bounds
+  kQuantDynamic = 1,    // fused amax + ring push + cast (current pass included)
+  kQuantRing = 2,       // cast with the layer's current ring scales, ring unchanged
+  kQuantAmaxOnly = 3,   // per-tensor amax into amax_out, nothing cast or pushed
 };
 
 cudaError_t launch_quantize(const QuantLaunch& q, cudaStream_t stream);

@@ -36,6 +36,8 @@ struct QuantArgs {
   int64_t T;              // expected cu[B]
   GlobalState* gs;
   LayerState* ls;
+  int cast_with_ring;     // static kernel: 1 = use the ring scales qs (kQuantRing)
+  float* amax_out;        // amax kernel: device float[3]
 };
 
 constexpr int kThreads = 512;
@@ -251,6 +253,10 @@ __global__ void __launch_bounds__(kThreads) quant_dynamic_kernel(QuantArgs a) {
   }
 }
 
+// One read-cast-store sweep with known scales: the static bounds (which then
+// become the layer's current scales), or the ring's current scales as left by
+// the last ring update (a shard of a head-sharded pass, whose amax was
+// reduced across ranks and pushed with fp8attn_amax_ring_update).
 template <bool kContig>
 __global__ void __launch_bounds__(kThreads) quant_static_kernel(QuantArgs a) {
   if (!seqlens_ok(a)) {
@@ -259,10 +265,45 @@ __global__ void __launch_bounds__(kThreads) quant_static_kernel(QuantArgs a) {
   }
   const int64_t T = __ldg(a.cu + a.B);
   const int64_t nvec = T * a.H * 16;
-  for (int t = 0; t < 3; ++t) cast_sweep<kContig>(a, t, nvec, a.ls->static_qs[t], false);
-  if (blockIdx.x == 0 && threadIdx.x < 3) {
+  const float* qs = a.cast_with_ring ? a.ls->qs : a.ls->static_qs;
+  for (int t = 0; t < 3; ++t) cast_sweep<kContig>(a, t, nvec, qs[t], false);
+  if (!a.cast_with_ring && blockIdx.x == 0 && threadIdx.x < 3) {
     a.ls->qs[threadIdx.x] = a.ls->static_qs[threadIdx.x];
     a.ls->ds[threadIdx.x] = a.ls->static_ds[threadIdx.x];
+  }
+}
+
+// Per-tensor amax only (no cast, ring untouched): every CTA folds its share
+// into the global amax words; the last CTA out writes the three values as
+// floats (NaN ignored, an infinite amax stays infinite) and clears the words.
+template <bool kContig>
+__global__ void __launch_bounds__(kThreads) quant_amax_kernel(QuantArgs a) {
+  __shared__ uint32_t red[kThreads / 32];
+  if (!seqlens_ok(a)) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(&a.gs->error, kErrSeqlens);
+    return;
+  }
+  const int64_t T = __ldg(a.cu + a.B);
+  const int64_t nvec = T * a.H * 16;
+  for (int t = 0; t < 3; ++t) {
+    uint32_t m = amax_sweep<kContig>(a, t, nvec);
+    m = block_max(m, red);
+    if (threadIdx.x == 0 && m != 0) atomicMax(&a.gs->amax_bits[t], m);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const uint32_t done = atomicAdd(&a.gs->done_count, 1u) + 1u;
+    if (done == gridDim.x) {
+      __threadfence();
+      for (int t = 0; t < 3; ++t) {
+        const uint32_t bits = *reinterpret_cast<volatile uint32_t*>(&a.gs->amax_bits[t]);
+        a.amax_out[t] = __uint_as_float(bits << 16);
+        a.gs->amax_bits[t] = 0;
+      }
+      a.gs->done_count = 0;
+      __threadfence();
+    }
   }
 }
 
@@ -332,6 +373,8 @@ cudaError_t launch_quantize(const QuantLaunch& q, cudaStream_t stream) {
   a.T = q.total_tokens;
   a.gs = static_cast<GlobalState*>(q.gs);
   a.ls = static_cast<LayerState*>(q.ls);
+  a.cast_with_ring = q.kind == kQuantRing;
+  a.amax_out = q.amax_out;
   const bool contig = q.src_seq_start == nullptr && q.head_stride == kHeadDim &&
                       q.tok_stride == static_cast<int64_t>(q.heads) * kHeadDim;
   // enough CTAs to cover the upper bound of the work, at most one full wave
@@ -343,7 +386,19 @@ cudaError_t launch_quantize(const QuantLaunch& q, cudaStream_t stream) {
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
-  if (q.dynamic) {
+  if (q.kind == kQuantAmaxOnly) {
+    // no grid-wide wait: any grid size works; one wave at most
+    const void* fn = contig ? reinterpret_cast<const void*>(&quant_amax_kernel<true>)
+                            : reinterpret_cast<const void*>(&quant_amax_kernel<false>);
+    const int cap = contig ? max_coresident(quant_amax_kernel<true>, kThreads)
+                           : max_coresident(quant_amax_kernel<false>, kThreads);
+    if (cap <= 0) return cudaErrorInvalidConfiguration;
+    cfg.gridDim = dim3(static_cast<int>(want < cap ? (want < 1 ? 1 : want) : cap));
+    cfg.attrs = nullptr;
+    cfg.numAttrs = 0;
+    return cudaLaunchKernelExC(&cfg, fn, args);
+  }
+  if (q.kind == kQuantDynamic) {
     const void* fn = contig ? reinterpret_cast<const void*>(&quant_dynamic_kernel<true>)
                             : reinterpret_cast<const void*>(&quant_dynamic_kernel<false>);
     const int cap = contig ? max_coresident(quant_dynamic_kernel<true>, kThreads)
@@ -633,6 +688,8 @@ int fp8attn_quantize_qkv_noalloc(const void* q, const void* k, const void* v, in
   a.T = total_tokens;
   a.gs = nullptr;
   a.ls = nullptr;
+  a.cast_with_ring = 0;
+  a.amax_out = nullptr;
   n.scratch = scratch;
   n.descale_out = d_descale_out;
   n.scale_out = d_scale_out;
