@@ -94,6 +94,17 @@ def test_host_argument_checks_need_no_gpu(L):
                                 None, None) == 0
     assert L.fp8attn_create(0, P(256), 1 << 20, None, ctypes.byref(P())) == 1
     assert L.fp8attn_e4m3_encode(None, 5, 1.0, None, None) == 1
+    # the amax-only entry point rejects a null context, a null output, a bad
+    # head_dim and misaligned sources before any CUDA call
+    f3 = P(256)
+    assert L.fp8attn_amax_qkv(None, P(16), P(16), P(16), 1024, 128, None, P(16), 1, 8, 8, 8,
+                              128, f3, None) == 1
+    assert L.fp8attn_amax_qkv(P(64), P(16), P(16), P(16), 1024, 128, None, P(16), 1, 8, 8, 8,
+                              128, None, None) == 1
+    assert L.fp8attn_amax_qkv(P(64), P(16), P(16), P(16), 1024, 128, None, P(16), 1, 8, 8, 8,
+                              64, f3, None) == 4
+    assert L.fp8attn_amax_qkv(P(64), P(17), P(16), P(16), 1024, 128, None, P(16), 1, 8, 8, 8,
+                              128, f3, None) == 4
     # the wait self-test checks its limit (0 < limit <= 1 s) and output first
     n = ctypes.c_int(0)
     assert L.fp8attn_selftest_bounded_waits(ctypes.c_uint64(0), ctypes.byref(n), None) == 1
