@@ -31,6 +31,9 @@ def _codes(T, H, seed, scale=1.0):
 CASES = [
     ([1], 1), ([5], 2), ([128], 1), ([129], 1), ([256], 2), ([257], 1), ([383], 3),
     ([1000, 17], 2), ([5, 300, 129], 3), ([64, 0, 200, 0], 2), ([513, 1, 255], 1),
+    # enough (sequence, head, 256-query block) units to fill whole waves of
+    # the GPU: ragged sequences through both the main and the tail kernel
+    ([257, 1, 129], 60), ([1000, 17], 40),
 ]
 
 
