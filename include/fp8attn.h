@@ -262,6 +262,25 @@ int fp8attn_select_mode_at_step(const fp8attn_ctx* ctx, const uint8_t* skip_laye
 fp8attn_status fp8attn_e4m3_encode(const float* d_in, int64_t n, float scale, void* d_out,
                                    void* stream);
 
+/* Head-group regrouping for sequence-parallel (Ulysses) attention
+ * (vLLM-Omni docs, "Quantized KV Cache", Configuration: the offline
+ * diffusion example shards the DiT's sequence over a Ulysses degree of 4).
+ * Each rank holds a contiguous slice of the tokens; an all-to-all gives every
+ * rank all tokens of num_heads/groups heads and a second one returns the
+ * attention output.  An all-to-all moves one contiguous chunk per rank, so:
+ *   to_groups = 1: d_src [tokens, num_heads, head_bytes] ->
+ *                  d_dst [groups, tokens, num_heads/groups, head_bytes]
+ *   to_groups = 0: the inverse ([groups, tokens, H/groups, hb] -> [tokens, H, hb]).
+ * head_bytes is the byte size of one head row (256 for bf16 with
+ * head_dim 128, 128 for E4M3 codes).  Device buffers, caller-owned, must not
+ * overlap.  Asynchronous on `stream`.  Errors: INVALID (negative tokens,
+ * groups < 1, num_heads not a multiple of groups, to_groups not 0/1, null or
+ * overlapping buffers), UNSUPPORTED (head_bytes not a multiple of 16, buffers
+ * not 16-byte aligned), CUDA.  tokens == 0 is a no-op. */
+fp8attn_status fp8attn_regroup_heads(const void* d_src, void* d_dst, int64_t tokens,
+                                    int num_heads, int groups, int head_bytes, int to_groups,
+                                    void* stream);
+
 /* Self-test of the bounded waits (failure detection without a GPU fault).
  * The pages have no counterpart: every wait inside this library's kernels
  * (mbarrier waits of the attention kernels, the grid barrier of the

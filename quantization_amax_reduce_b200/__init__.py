@@ -14,6 +14,7 @@ prefix.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import json
 import math
@@ -27,7 +28,8 @@ __all__ = [
     "DYNAMIC", "STATIC", "SKIP", "RING_LENGTH", "DEFAULT_MARGIN", "FP8AttnError", "lib",
     "Context", "varlen_fwd", "varlen_fwd_bf16", "parse_selector", "e4m3_encode",
     "launch_count", "load_scale_file", "save_scale_file", "read_error_word",
-    "quantize_qkv_noalloc", "quantize_qkv_noalloc_error",
+    "quantize_qkv_noalloc", "quantize_qkv_noalloc_error", "RING",
+    "head_sharded_dynamic_quantize", "regroup_heads", "TorchComm", "ulysses_attention",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -97,6 +99,7 @@ def lib() -> ctypes.CDLL:
                                              P, P]),
         "fp8attn_quantize_qkv_noalloc_error": (I, [P]),
         "fp8attn_selftest_bounded_waits": (I, [ctypes.c_uint64, ctypes.POINTER(I), P]),
+        "fp8attn_regroup_heads": (I, [P, P, I64, I, I, I, I, P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -534,3 +537,139 @@ def head_sharded_dynamic_quantize(ctx: "Context", layer: int, q: torch.Tensor, k
             dist.all_reduce(amax, op=dist.ReduceOp.MAX, group=group)
     ctx.amax_ring_update(layer, amax, stream=stream)
     return ctx.quantize_qkv(layer, RING, q, k, v, cu_seqlens, max_seqlen, out=out, stream=stream)
+
+
+def regroup_heads(x: torch.Tensor, groups: int, to_groups: bool = True,
+                  out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Head-group regrouping around the all-to-all of sequence-parallel
+    attention: [T, H, 128] -> [groups, T, H/groups, 128] (``to_groups``) or
+    back.  bf16 or uint8 (E4M3 codes), contiguous, on the device."""
+    _require_cuda(x, "x")
+    if x.dtype not in (torch.bfloat16, torch.uint8) or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bf16 or uint8 tensor")
+    groups = int(groups)
+    if to_groups:
+        if x.dim() != 3 or x.shape[-1] != HEAD_DIM:
+            raise ValueError("x must be [T, H, 128]")
+        T, H, _ = x.shape
+        if groups < 1 or H % groups:
+            raise ValueError("num_heads must be a multiple of groups")
+        shape = (groups, T, H // groups, HEAD_DIM)
+    else:
+        if x.dim() != 4 or x.shape[0] != groups or x.shape[-1] != HEAD_DIM:
+            raise ValueError("x must be [groups, T, H/groups, 128]")
+        _, T, Hn, _ = x.shape
+        H = groups * Hn
+        shape = (T, H, HEAD_DIM)
+    if out is None:
+        out = torch.empty(shape, dtype=x.dtype, device=x.device)
+    elif tuple(out.shape) != shape or out.dtype != x.dtype or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous {shape} {x.dtype} tensor")
+    _check(lib().fp8attn_regroup_heads(_ptr(x), _ptr(out), T, H, groups,
+                                       HEAD_DIM * x.element_size(), int(bool(to_groups)),
+                                       ctypes.c_void_p(_stream(stream, x.device))),
+           "fp8attn_regroup_heads")
+    return out
+
+
+class TorchComm:
+    """The exchanges of the sharded paths over a torch.distributed process
+    group (NCCL between GPUs).  Without an initialised process group it is a
+    single rank and exchanges nothing."""
+
+    def __init__(self, group=None):
+        import torch.distributed as dist
+        self._dist = dist
+        self.group = group
+        self._on = dist.is_available() and dist.is_initialized()
+
+    def size(self) -> int:
+        return self._dist.get_world_size(self.group) if self._on else 1
+
+    def rank(self) -> int:
+        return self._dist.get_rank(self.group) if self._on else 0
+
+    def all_reduce_max(self, t: torch.Tensor) -> None:
+        if self.size() > 1:
+            self._dist.all_reduce(t, op=self._dist.ReduceOp.MAX, group=self.group)
+
+    def all_to_all(self, out: torch.Tensor, inp: torch.Tensor) -> None:
+        """Chunk i of ``inp`` (split along dim 0) goes to rank i; chunk i of
+        ``out`` comes from rank i."""
+        self._dist.all_to_all_single(out, inp, group=self.group)
+
+
+def ulysses_attention(ctx: "Context", layer: int, mode: int, q: torch.Tensor, k: torch.Tensor,
+                      v: torch.Tensor, comm=None, softmax_scale: float = 0.0,
+                      stream=None) -> torch.Tensor:
+    """Sequence-parallel (Ulysses) attention over one sequence whose tokens are
+    split evenly across the ranks of ``comm`` (a :class:`TorchComm` by
+    default): rank r holds tokens [r S_loc, (r+1) S_loc) of Q, K, V as bf16
+    [S_loc, H, 128]; it returns the same tokens of the output, bf16
+    [S_loc, H, 128].  vLLM-Omni docs, "Quantized KV Cache", Configuration:
+    the offline diffusion example shards the DiT over a Ulysses degree of 4.
+
+    FP8 modes quantise BEFORE the exchange, so the all-to-all moves 1-byte
+    codes: DYNAMIC takes the amax of this rank's tokens (all heads), the
+    all-reduce MAX of the three values makes it the amax of the whole
+    sequence, the ring is updated, and each group of H/n heads is cast with
+    the ring scales straight into its send chunk; STATIC casts with the
+    layer's static bounds.  Then: all-to-all (rank r receives every rank's
+    tokens of head group r, i.e. the whole sequence in token order), attention
+    on those heads, the return all-to-all, and the inverse head regrouping.
+    SKIP regroups and exchanges bf16 and runs the bf16 attention.  Codes,
+    scales, ring and output equal one single-GPU pass over the whole sequence
+    (``quantize_qkv`` with the same mode, then ``varlen_fwd``).  Every rank
+    must make the same calls in the same order."""
+    comm = TorchComm() if comm is None else comm
+    n = int(comm.size())
+    if q.dim() != 3 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must be [S_local, H, 128] of the same shape")
+    if mode not in (DYNAMIC, STATIC, SKIP):
+        raise ValueError("mode must be DYNAMIC, STATIC or SKIP")
+    S_loc, H, D = q.shape
+    if D != HEAD_DIM:
+        raise ValueError("head_dim must be 128")
+    if H % n:
+        raise ValueError("num_heads must be a multiple of the number of ranks")
+    Hn, S = H // n, S_loc * n
+    dev = q.device
+    cm = torch.cuda.stream(stream if isinstance(stream, torch.cuda.Stream)
+                           else torch.cuda.ExternalStream(int(stream))) \
+        if stream is not None else contextlib.nullcontext()
+    with cm:
+        cu_loc = _cu_tensor([0, S_loc], dev)
+        cu_all = _cu_tensor([0, S], dev)
+        if mode == SKIP:
+            send = [regroup_heads(x.contiguous(), n) if n > 1 else x.contiguous()
+                    for x in (q, k, v)]
+        else:
+            cast = STATIC
+            if mode == DYNAMIC:
+                amax = ctx.amax_qkv(q, k, v, cu_loc, S_loc)
+                comm.all_reduce_max(amax)
+                ctx.amax_ring_update(layer, amax)
+                cast = RING
+            send = [torch.empty((n, S_loc, Hn, D), dtype=torch.uint8, device=dev)
+                    for _ in range(3)]
+            for g in range(n):
+                h = slice(g * Hn, (g + 1) * Hn)
+                ctx.quantize_qkv(layer, cast, q[:, h], k[:, h], v[:, h], cu_loc, S_loc,
+                                 out=(send[0][g], send[1][g], send[2][g]))
+        if n > 1:
+            recv = [torch.empty_like(x) for x in send]
+            for r, x in zip(recv, send):
+                comm.all_to_all(r, x)
+        else:
+            recv = send
+        recv = [x.view(S, Hn, D) for x in recv]
+        if mode == SKIP:
+            o = varlen_fwd_bf16(recv[0], recv[1], recv[2], cu_all, S, softmax_scale)
+        else:
+            o = varlen_fwd(recv[0], recv[1], recv[2], cu_all, S, ctx.descale_ptr(layer),
+                           softmax_scale)
+        if n == 1:
+            return o.view(S_loc, H, D)
+        back = torch.empty_like(o)
+        comm.all_to_all(back, o)
+        return regroup_heads(back.view(n, S_loc, Hn, D), n, to_groups=False)

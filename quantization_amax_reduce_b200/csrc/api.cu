@@ -485,6 +485,26 @@ fp8attn_status fp8attn_e4m3_encode(const float* d_in, int64_t n, float scale, vo
   return FP8ATTN_OK;
 }
 
+fp8attn_status fp8attn_regroup_heads(const void* d_src, void* d_dst, int64_t tokens,
+                                    int num_heads, int groups, int head_bytes, int to_groups,
+                                    void* stream) {
+  if (tokens < 0 || num_heads < 1 || groups < 1 || head_bytes < 1) return FP8ATTN_ERR_INVALID;
+  if (num_heads % groups) return FP8ATTN_ERR_INVALID;
+  if (to_groups != 0 && to_groups != 1) return FP8ATTN_ERR_INVALID;
+  if (head_bytes % 16) return FP8ATTN_ERR_UNSUPPORTED;
+  if (tokens == 0) return FP8ATTN_OK;
+  if (!d_src || !d_dst) return FP8ATTN_ERR_INVALID;
+  if (!aligned(d_src, 16) || !aligned(d_dst, 16)) return FP8ATTN_ERR_UNSUPPORTED;
+  const uintptr_t bytes = static_cast<uintptr_t>(tokens) * num_heads * head_bytes;
+  const uintptr_t s0 = reinterpret_cast<uintptr_t>(d_src), d0 = reinterpret_cast<uintptr_t>(d_dst);
+  if (s0 < d0 + bytes && d0 < s0 + bytes) return FP8ATTN_ERR_INVALID;   // overlap
+  const cudaError_t e = launch_regroup_heads(d_src, d_dst, tokens, num_heads, groups, head_bytes,
+                                             to_groups, as_stream(stream));
+  if (e != cudaSuccess) return FP8ATTN_ERR_CUDA;
+  g_launches.fetch_add(1);
+  return FP8ATTN_OK;
+}
+
 uint64_t fp8attn_launch_count(void) { return g_launches.load(); }
 
 }  // extern "C"

@@ -49,4 +49,9 @@ struct AttnLaunch {
 
 cudaError_t launch_attention(const AttnLaunch& p, int64_t total_tokens, cudaStream_t stream);
 
+// [T, H, hb] <-> [G, T, H/G, hb] (to_groups = 1 / 0); hb a multiple of 16,
+// H a multiple of G, 16-byte aligned, non-overlapping buffers.
+cudaError_t launch_regroup_heads(const void* src, void* dst, int64_t tokens, int heads,
+                                 int groups, int head_bytes, int to_groups, cudaStream_t stream);
+
 }  // namespace fp8attn

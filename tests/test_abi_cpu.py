@@ -110,6 +110,18 @@ def test_host_argument_checks_need_no_gpu(L):
     assert L.fp8attn_selftest_bounded_waits(ctypes.c_uint64(0), ctypes.byref(n), None) == 1
     assert L.fp8attn_selftest_bounded_waits(ctypes.c_uint64(2 * 10**9), ctypes.byref(n), None) == 1
     assert L.fp8attn_selftest_bounded_waits(ctypes.c_uint64(10**6), None, None) == 1
+    # head regrouping: sizes, groups, direction, alignment and overlap are
+    # checked on the host; zero tokens is a no-op
+    src, dst = P(1 << 20), P(1 << 24)
+    assert L.fp8attn_regroup_heads(src, dst, -1, 8, 2, 256, 1, None) == 1
+    assert L.fp8attn_regroup_heads(src, dst, 64, 8, 3, 256, 1, None) == 1    # 8 % 3
+    assert L.fp8attn_regroup_heads(src, dst, 64, 8, 0, 256, 1, None) == 1
+    assert L.fp8attn_regroup_heads(src, dst, 64, 8, 2, 256, 2, None) == 1    # direction
+    assert L.fp8attn_regroup_heads(None, dst, 64, 8, 2, 256, 1, None) == 1
+    assert L.fp8attn_regroup_heads(src, P((1 << 20) + 4096), 64, 8, 2, 256, 1, None) == 1
+    assert L.fp8attn_regroup_heads(src, dst, 64, 8, 2, 100, 1, None) == 4    # 100 % 16
+    assert L.fp8attn_regroup_heads(P((1 << 20) + 8), dst, 64, 8, 2, 256, 1, None) == 4
+    assert L.fp8attn_regroup_heads(None, None, 0, 8, 2, 256, 0, None) == 0
 
 
 def test_scale_file_round_trip(tmp_path, golden_dir):
