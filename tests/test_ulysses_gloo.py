@@ -207,3 +207,28 @@ def test_ulysses_ranks_equal_one_pass_over_the_whole_sequence(world):
             if ds is not None:
                 assert g_ds == ds, (kind, p, rank)
             assert g_slots == slots, (kind, p, rank)
+
+
+class _FakeComm:
+    def __init__(self, n):
+        self.n = n
+
+    def size(self):
+        return self.n
+
+    def rank(self):
+        return 0
+
+
+def test_argument_checks_before_any_exchange():
+    import quantization_amax_reduce_b200 as qar
+    x = torch.zeros(8, 4, D, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="multiple of the number of ranks"):
+        qar.ulysses_attention(None, 0, qar.DYNAMIC, x, x, x, comm=_FakeComm(3))
+    with pytest.raises(ValueError, match="mode"):
+        qar.ulysses_attention(None, 0, qar.RING, x, x, x, comm=_FakeComm(2))
+    with pytest.raises(ValueError, match="same shape"):
+        qar.ulysses_attention(None, 0, qar.DYNAMIC, x, x[:4], x, comm=_FakeComm(2))
+    with pytest.raises(ValueError, match="head_dim"):
+        y = torch.zeros(8, 4, 64, dtype=torch.bfloat16)
+        qar.ulysses_attention(None, 0, qar.DYNAMIC, y, y, y, comm=_FakeComm(2))
