@@ -599,6 +599,20 @@ class TorchComm:
         self._dist.all_to_all_single(out, inp, group=self.group)
 
 
+_SINGLE_SEQ_CU: Dict[Tuple[str, int], torch.Tensor] = {}
+
+
+def _single_seq_cu(S: int, device) -> torch.Tensor:
+    """Device cu_seqlens [0, S], made once per (device, S): later calls copy
+    nothing from the host, so they can be captured in a CUDA graph."""
+    key = (str(torch.device(device)), int(S))
+    t = _SINGLE_SEQ_CU.get(key)
+    if t is None:
+        t = _cu_tensor([0, int(S)], device)
+        _SINGLE_SEQ_CU[key] = t
+    return t
+
+
 def ulysses_attention(ctx: "Context", layer: int, mode: int, q: torch.Tensor, k: torch.Tensor,
                       v: torch.Tensor, comm=None, softmax_scale: float = 0.0,
                       stream=None) -> torch.Tensor:
@@ -638,8 +652,8 @@ def ulysses_attention(ctx: "Context", layer: int, mode: int, q: torch.Tensor, k:
                            else torch.cuda.ExternalStream(int(stream))) \
         if stream is not None else contextlib.nullcontext()
     with cm:
-        cu_loc = _cu_tensor([0, S_loc], dev)
-        cu_all = _cu_tensor([0, S], dev)
+        cu_loc = _single_seq_cu(S_loc, dev)
+        cu_all = _single_seq_cu(S, dev)
         if mode == SKIP:
             send = [regroup_heads(x.contiguous(), n) if n > 1 else x.contiguous()
                     for x in (q, k, v)]
