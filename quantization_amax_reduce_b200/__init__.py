@@ -520,21 +520,24 @@ def selftest_bounded_waits(mbar_limit_ns: int = 50_000_000, device=None) -> int:
 
 def head_sharded_dynamic_quantize(ctx: "Context", layer: int, q: torch.Tensor, k: torch.Tensor,
                                   v: torch.Tensor, cu_seqlens, max_seqlen: int, group=None,
-                                  out: Optional[Sequence[torch.Tensor]] = None, stream=None
-                                  ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+                                  out: Optional[Sequence[torch.Tensor]] = None, stream=None,
+                                  comm=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """One dynamic pass over this rank's heads of a layer whose heads are
     sharded across the ranks of `group` (torch.distributed, NCCL on GPUs):
     local amax -> all-reduce MAX of the three values (the only exchange) ->
     push into this rank's ring -> cast this shard with the ring scales.  Every
     rank ends with the ring, scales and codes one DYNAMIC pass over all heads
     would give.  With no process group (or one rank) it is the same sequence
-    without the all-reduce."""
-    import torch.distributed as dist
+    without the all-reduce.  The exchange goes through ``comm`` (default: a
+    :class:`TorchComm` over ``group``)."""
+    comm = TorchComm(group) if comm is None else comm
     amax = ctx.amax_qkv(q, k, v, cu_seqlens, max_seqlen, stream=stream)
-    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
-        s = torch.cuda.current_stream(q.device) if stream is None else stream
-        with torch.cuda.stream(s if isinstance(s, torch.cuda.Stream) else torch.cuda.ExternalStream(int(s))):
-            dist.all_reduce(amax, op=dist.ReduceOp.MAX, group=group)
+    if comm.size() > 1:
+        cm = torch.cuda.stream(stream if isinstance(stream, torch.cuda.Stream)
+                               else torch.cuda.ExternalStream(int(stream))) \
+            if stream is not None else contextlib.nullcontext()
+        with cm:
+            comm.all_reduce_max(amax)
     ctx.amax_ring_update(layer, amax, stream=stream)
     return ctx.quantize_qkv(layer, RING, q, k, v, cu_seqlens, max_seqlen, out=out, stream=stream)
 

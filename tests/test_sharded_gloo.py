@@ -1,7 +1,8 @@
-"""Head-sharded dynamic quantisation on two gloo ranks (CPU), with the oracle
-standing in for each rank's kernels: the per-tensor amax is the only value
-that crosses ranks (an all-reduce MAX of three floats), after which every
-rank's ring, scales and codes equal those of one pass over all heads.
+"""Head-sharded dynamic quantisation on two gloo ranks (CPU): the product's
+``head_sharded_dynamic_quantize`` runs its real all-reduce (MAX of three
+floats, through ``TorchComm`` over gloo) with the oracle standing in for each
+rank's kernels.  After it every rank's ring, scales and codes equal those of
+one pass over all heads.
 
 vLLM docs, "FP8 ViT encoder attention", usage: scales come from a ring of
 observed Q/K/V amax values; the amax is a max over the whole tensor, so a
@@ -28,40 +29,38 @@ def _free_port():
 
 
 def _inputs(p):
-    """bf16 bit patterns [T, H, D] for pass p, with one large channel on a
-    head of the second shard so the shards' amax differ."""
+    """bf16 [T, H, D] tensors for pass p, with one large channel on a head of
+    the second shard so the shards' amax differ."""
     import synthetic
     q, k, v, cu = synthetic.small_qkv(500 + p, LENS, H=H, scale=1.0 + p)
     out = []
     for x in (q, k, v):
         x = x.clone()
         x[:, H - 1, 3] *= 8.0
-        out.append(synthetic.bf16_bits(x))
+        out.append(x)
     return out, cu
 
 
 def _worker(rank, world, port, q):
     import sys
-    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
-    import oracle
+    here = os.path.dirname(os.path.abspath(__file__))
+    sys.path[:0] = [os.path.dirname(here), here]
+    import quantization_amax_reduce_b200 as qar
+    from oracle_context import OracleContext
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         hs = H // world
         heads = slice(rank * hs, (rank + 1) * hs)
-        rings = [oracle.Ring() for _ in range(3)]
+        ctx = OracleContext()
         results = []
         for p in range(PASSES):
-            bits, cu = _inputs(p)
-            shard = [np.ascontiguousarray(b[:, heads, :]) for b in bits]
-            local = torch.tensor([oracle.amax(x, cu, hs, D)[0] for x in shard], dtype=torch.float32)
-            dist.all_reduce(local, op=dist.ReduceOp.MAX)
-            codes, scales = [], []
-            for t in range(3):
-                qs, ds = rings[t].dynamic_step(float(local[t]), False)
-                scales.append((float(qs), float(ds)))
-                codes.append(oracle.quantize(shard[t], cu, hs, D, qs))
-            results.append((scales, [c.tobytes() for c in codes], [r.slots.tolist() for r in rings]))
+            x, cu = _inputs(p)
+            shard = [t[:, heads, :] for t in x]          # strided views, as on a GPU
+            codes = qar.head_sharded_dynamic_quantize(ctx, 0, *shard, cu, max(LENS))
+            scales = [(float(a), float(b)) for a, b in zip(ctx.qs, ctx.ds)]
+            results.append((scales, [c.numpy().tobytes() for c in codes],
+                            [r.slots.tolist() for r in ctx.rings]))
         q.put((rank, results))
     finally:
         dist.destroy_process_group()
@@ -69,6 +68,7 @@ def _worker(rank, world, port, q):
 
 def test_two_rank_head_sharded_pass_equals_the_unsharded_pass():
     import oracle
+    import synthetic
     world = 2
     port = _free_port()
     ctx = mp.get_context("spawn")
@@ -95,7 +95,8 @@ def test_two_rank_head_sharded_pass_equals_the_unsharded_pass():
     rings = [oracle.Ring() for _ in range(3)]
     hs = H // world
     for p in range(PASSES):
-        bits, cu = _inputs(p)
+        x, cu = _inputs(p)
+        bits = [synthetic.bf16_bits(t) for t in x]
         for t in range(3):
             a, nf = oracle.amax(bits[t], cu, H, D)
             qs, ds = rings[t].dynamic_step(a, nf)

@@ -47,49 +47,6 @@ def _inputs(p):
     return q, k, v
 
 
-class OracleContext:
-    """One layer's ring and scales, with the oracle doing each step."""
-
-    def __init__(self):
-        import oracle
-        self.o = oracle
-        self.rings = [oracle.Ring() for _ in range(3)]
-        self.qs = [np.float32(1.0)] * 3
-        self.ds = [np.float32(1.0)] * 3
-        self.static = None
-
-    def amax_qkv(self, q, k, v, cu, max_seqlen):
-        import synthetic
-        vals = []
-        for x in (q, k, v):
-            a, nf = self.o.amax(synthetic.bf16_bits(x.contiguous()), np.asarray(cu), x.shape[1], D)
-            vals.append(float("inf") if nf else float(a))
-        return torch.tensor(vals, dtype=torch.float32)
-
-    def amax_ring_update(self, layer, amax):
-        for t in range(3):
-            a = float(amax[t])
-            self.qs[t], self.ds[t] = self.rings[t].dynamic_step(0.0 if np.isinf(a) else a,
-                                                                bool(np.isinf(a)))
-
-    def quantize_qkv(self, layer, mode, q, k, v, cu, max_seqlen, out):
-        import synthetic
-        from quantization_amax_reduce_b200 import RING, STATIC
-        if mode == STATIC:
-            sc = [self.o.scales_from_bound(np.float32(a)) for a in self.static]
-            self.qs = [s[0] for s in sc]
-            self.ds = [s[1] for s in sc]
-        else:
-            assert mode == RING
-        for t, x in enumerate((q, k, v)):
-            codes = self.o.quantize(synthetic.bf16_bits(x.contiguous()), np.asarray(cu),
-                                    x.shape[1], D, self.qs[t])
-            out[t].copy_(torch.from_numpy(codes))
-
-    def descale_ptr(self, layer):
-        return [float(d) for d in self.ds]
-
-
 def _oracle_kernels(qar):
     """Stand-ins for the attention and regroup kernels (this process only)."""
     import oracle
@@ -117,14 +74,15 @@ def _oracle_kernels(qar):
 
 def _worker(rank, world, port, out_q):
     import sys
-    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    here = os.path.dirname(os.path.abspath(__file__))
+    sys.path[:0] = [os.path.dirname(here), here]
     import quantization_amax_reduce_b200 as qar
     _oracle_kernels(qar)
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        ctx = OracleContext()
-        ctx.static = STATIC_VALUES
+        from oracle_context import OracleContext
+        ctx = OracleContext(STATIC_VALUES)
         comm = qar.TorchComm()
         assert comm.size() == world and comm.rank() == rank
         S_loc = S_TOTAL // world
