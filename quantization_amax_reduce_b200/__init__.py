@@ -153,6 +153,18 @@ def _qkv_source(q, k, v, cu_seqlens, total_tokens, src_seq_start):
     return H, tok_stride, head_stride, cu, B, total_tokens, sss
 
 
+def _check_out(t, name: str, dtype, numel: int, device) -> None:
+    """A caller-provided output: contiguous, on the inputs' device, of the
+    right dtype and large enough that no kernel writes past its end."""
+    _require_cuda(t, name)
+    if t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor")
+    if t.device != torch.device(device):
+        raise ValueError(f"{name} must be on {device}")
+    if t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} elements, {numel} needed")
+
+
 def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -214,6 +226,11 @@ class Context:
         if out is None:
             out = [torch.empty((total_tokens, H, HEAD_DIM), dtype=torch.uint8, device=q.device)
                    for _ in range(3)]
+        else:
+            if len(out) != 3:
+                raise ValueError("out must hold three tensors (q8, k8, v8)")
+            for name, t in zip(("q8", "k8", "v8"), out):
+                _check_out(t, name, torch.uint8, int(total_tokens) * H * HEAD_DIM, q.device)
         _check(lib().fp8attn_quantize_qkv(
             self._h, layer, mode, _ptr(q), _ptr(k), _ptr(v), tok_stride, head_stride, _ptr(sss),
             _ptr(cu), B, int(max_seqlen), int(total_tokens), H, HEAD_DIM, _ptr(out[0]),
@@ -231,6 +248,8 @@ class Context:
             q, k, v, cu_seqlens, total_tokens, src_seq_start)
         if out is None:
             out = torch.empty(3, dtype=torch.float32, device=q.device)
+        else:
+            _check_out(out, "out", torch.float32, 3, q.device)
         _check(lib().fp8attn_amax_qkv(
             self._h, _ptr(q), _ptr(k), _ptr(v), tok_stride, head_stride, _ptr(sss), _ptr(cu), B,
             int(max_seqlen), int(total_tokens), H, HEAD_DIM, _ptr(out),
@@ -349,6 +368,8 @@ def _attn_common(q, k, v, cu_seqlens, out, dtype):
     cu = _cu_tensor(cu_seqlens, q.device)
     if out is None:
         out = torch.empty((T, H, HEAD_DIM), dtype=torch.bfloat16, device=q.device)
+    else:
+        _check_out(out, "out", torch.bfloat16, T * H * HEAD_DIM, q.device)
     return T, H, cu, out
 
 
@@ -457,6 +478,8 @@ def quantize_qkv_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_s
         if src_seq_start is not None:
             raise ValueError("total_tokens is required with a padded source")
         total_tokens = q.shape[-3] if q.dim() == 3 else q.shape[0] * q.shape[1]
+    for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        _check_out(t, name, torch.uint8, int(total_tokens) * H * HEAD_DIM, q.device)
     sss = None if src_seq_start is None else _cu_tensor(src_seq_start, q.device)
     _check(lib().fp8attn_quantize_qkv_noalloc(
         _ptr(q), _ptr(k), _ptr(v), q.stride(-3), q.stride(-2), _ptr(sss), _ptr(cu),
