@@ -143,10 +143,13 @@ def _qkv_source(q, k, v, cu_seqlens, total_tokens, src_seq_start):
     head_stride, tok_stride = q.stride(-2), q.stride(-3)
     cu = _cu_tensor(cu_seqlens, q.device)
     B = cu.numel() - 1
+    rows = q.shape[-3] if q.dim() == 3 else q.shape[0] * q.shape[1]
     if total_tokens is None:
         if src_seq_start is not None:
             raise ValueError("total_tokens is required with a padded source")
-        total_tokens = q.shape[-3] if q.dim() == 3 else q.shape[0] * q.shape[1]
+        total_tokens = rows
+    elif src_seq_start is None and int(total_tokens) > rows:
+        raise ValueError(f"total_tokens {total_tokens} exceeds the {rows} source rows")
     sss = None
     if src_seq_start is not None:
         sss = _cu_tensor(src_seq_start, q.device)

@@ -42,5 +42,7 @@ def test_output_buffers_are_checked_before_launch():
     ds = torch.zeros(3, dtype=torch.float32, device=DEV)
     with pytest.raises(ValueError, match="needed"):
         qar.quantize_qkv_noalloc(q, k, v, cu_d, 100, *small, ds)
+    with pytest.raises(ValueError, match="source rows"):
+        ctx.quantize_qkv(0, qar.DYNAMIC, q, k, v, cu_d, 100, total_tokens=129)
     # only the one good quantisation launched
     assert n1 == n0 + 1 and qar.launch_count() == n1
