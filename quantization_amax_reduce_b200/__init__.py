@@ -505,10 +505,18 @@ def launch_count() -> int:
 _ALIASES = {"q": ("q", "q_scale"), "k": ("k", "k_scale"), "v": ("v", "v_scale")}
 
 
-def load_scale_file(path: str) -> Dict[str, Tuple[float, float, float]]:
+def load_scale_file(path: str, margin: float = 1.0) -> Dict[str, Tuple[float, float, float]]:
     """Read a per-layer {"q","k","v"} scale map (``q_scale``/``k_scale``/
     ``v_scale`` accepted as aliases), as in the vLLM FP8 ViT page's scale
-    file format section."""
+    file format section.
+
+    The page applies its save margin when the file is written, so by default
+    the values are used as stored (``margin=1.0``).  A file written without
+    the margin can be read with it applied here: each value becomes
+    fl32(value * margin)."""
+    margin = np.float32(margin)
+    if not np.isfinite(margin) or margin <= 0:
+        raise ValueError("margin must be a positive finite number")
     with open(path) as f:
         raw = json.load(f)
     out = {}
@@ -518,7 +526,7 @@ def load_scale_file(path: str) -> Dict[str, Tuple[float, float, float]]:
             keys = [k for k in _ALIASES[t] if k in entry]
             if not keys:
                 raise ValueError(f"layer {name!r} has no {t} value")
-            vals.append(float(entry[keys[0]]))
+            vals.append(float(np.float32(entry[keys[0]]) * margin))
         out[name] = tuple(vals)
     return out
 

@@ -138,3 +138,23 @@ def test_scale_file_round_trip(tmp_path, golden_dir):
     out = tmp_path / "saved.json"
     qar.save_scale_file(str(out), ["a", "b"], np.array([[1.5, 3.0, 4.5], [6.0, 7.5, 9.0]]))
     assert qar.load_scale_file(str(out)) == {"a": (1.5, 3.0, 4.5), "b": (6.0, 7.5, 9.0)}
+
+
+def test_scale_file_margin_on_load(tmp_path, golden_dir):
+    """The alternative reading of the static values (margin applied when the
+    file is read, not when it was written): each value becomes
+    fl32(value * margin); the default leaves the stored values as they are."""
+    import quantization_amax_reduce_b200 as qar
+    g = json.load(open(os.path.join(golden_dir, "static_scale_file.json")))
+    p = tmp_path / "scales.json"
+    p.write_text(json.dumps(g["map"]))
+    m = qar.load_scale_file(str(p), margin=1.5)
+    assert m["visual.blocks.0.attn.attn"] == (336.0, 297.0, 315.0)
+    p2 = tmp_path / "odd.json"
+    p2.write_text(json.dumps({"x": {"q": 0.1, "k": 3.0, "v": 1e-3}}))
+    got = qar.load_scale_file(str(p2), margin=1.5)["x"]
+    want = tuple(float(np.float32(np.float32(v) * np.float32(1.5))) for v in (0.1, 3.0, 1e-3))
+    assert got == want
+    for bad in (0.0, -1.0, float("inf"), float("nan")):
+        with pytest.raises(ValueError):
+            qar.load_scale_file(str(p), margin=bad)
