@@ -213,6 +213,25 @@ def oracle_sample(n_rows: int, quant_tokens: int, seed: int = 0):
     return (t1 - t0) + (t3 - t2), 4.0 * n_rows * S * D * H, 3 * quant_tokens * H * D, threads
 
 
+def host_cpu_info() -> dict:
+    """The host CPU the oracle ran on: model name and the cores this process
+    may run on (the oracle starts one thread per online core)."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        usable = os.cpu_count() or 1
+    return {"cpu_model": model, "usable_cores": usable}
+
+
 def cpu_baseline_full_step_estimate():
     """Oracle time for one full step, from a bounded sample: full quantisation
     of Q/K/V plus attention for 32 of the 8192 query rows (x256)."""
@@ -241,6 +260,7 @@ def cpu_baseline_full_step_estimate():
         "sample": (f"full static quantisation of Q/K/V ({t1 - t0:.2f} s) + fp64 attention of "
                    f"{n_rows}/{S} query rows x {H} heads ({t2 - t1:.2f} s, scaled x{S // n_rows})"),
         "seconds_per_step": step_s,
+        **host_cpu_info(),
     }
 
 
@@ -272,7 +292,7 @@ def run_reference(args):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD, "S": S, "heads": H, "head_dim": D},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, **host_cpu_info()},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
