@@ -139,11 +139,20 @@ def _qkv_source(q, k, v, cu_seqlens, total_tokens, src_seq_start):
         raise ValueError("q, k, v must share shape and strides")
     if q.shape[-1] != HEAD_DIM or q.stride(-1) != 1:
         raise ValueError("head_dim must be 128 and contiguous")
+    if q.dim() not in (3, 4):
+        raise ValueError("sources are [T, H, 128] or [B, S_max, H, 128]")
+    if q.dim() == 4 and q.shape[0] > 1 and q.stride(0) != q.shape[1] * q.stride(1):
+        # the kernels address row r of a padded source at r * tok_stride
+        raise ValueError("a padded source needs its sequences back to back "
+                         "(stride(0) == S_max * stride(1))")
     H = q.shape[-2]
     head_stride, tok_stride = q.stride(-2), q.stride(-3)
+    rows = q.shape[-3] if q.dim() == 3 else q.shape[0] * q.shape[1]
+    if src_seq_start is not None and not isinstance(src_seq_start, torch.Tensor) and \
+            not isinstance(cu_seqlens, torch.Tensor):
+        _check_padded_rows(cu_seqlens, src_seq_start, rows)
     cu = _cu_tensor(cu_seqlens, q.device)
     B = cu.numel() - 1
-    rows = q.shape[-3] if q.dim() == 3 else q.shape[0] * q.shape[1]
     if total_tokens is None:
         if src_seq_start is not None:
             raise ValueError("total_tokens is required with a padded source")
@@ -154,6 +163,22 @@ def _qkv_source(q, k, v, cu_seqlens, total_tokens, src_seq_start):
     if src_seq_start is not None:
         sss = _cu_tensor(src_seq_start, q.device)
     return H, tok_stride, head_stride, cu, B, total_tokens, sss
+
+
+def _check_padded_rows(cu_seqlens, src_seq_start, rows: int) -> None:
+    """Host-side check of a padded source given as host arrays: sequence b's
+    rows [src_seq_start[b], src_seq_start[b] + len_b) lie inside the source's
+    ``rows`` rows.  (Device tensors are not read back; the kernels take them
+    as given.)"""
+    cu = np.asarray(cu_seqlens, dtype=np.int64).ravel()
+    start = np.asarray(src_seq_start, dtype=np.int64).ravel()
+    if start.size != cu.size - 1:
+        raise ValueError("src_seq_start needs one entry per sequence")
+    lens = np.diff(cu)
+    if (lens < 0).any():
+        raise ValueError("cu_seqlens must not decrease")
+    if (start < 0).any() or (start + lens > rows).any():
+        raise ValueError(f"a sequence of the padded source lies outside its {rows} rows")
 
 
 def _check_out(t, name: str, dtype, numel: int, device) -> None:
@@ -464,6 +489,12 @@ def quantize_qkv_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_s
             raise ValueError(f"{name} must be bfloat16")
     if q.stride() != k.stride() or q.stride() != v.stride() or q.shape[-1] != HEAD_DIM:
         raise ValueError("q, k, v must share strides and have head_dim 128")
+    if q.shape != k.shape or q.shape != v.shape or q.stride(-1) != 1 or q.dim() not in (3, 4):
+        raise ValueError("q, k, v must be [T, H, 128] or [B, S_max, H, 128] with the channel "
+                         "contiguous")
+    if q.dim() == 4 and q.shape[0] > 1 and q.stride(0) != q.shape[1] * q.stride(1):
+        raise ValueError("a padded source needs its sequences back to back "
+                         "(stride(0) == S_max * stride(1))")
     for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
         _require_cuda(t, name)
         if t.dtype != torch.uint8 or not t.is_contiguous():

@@ -158,3 +158,19 @@ def test_scale_file_margin_on_load(tmp_path, golden_dir):
     for bad in (0.0, -1.0, float("inf"), float("nan")):
         with pytest.raises(ValueError):
             qar.load_scale_file(str(p), margin=bad)
+
+
+def test_padded_source_rows_checked_on_the_host():
+    """A padded source given with host-side cu_seqlens / src_seq_start is
+    checked before any launch: every sequence's rows lie inside the source."""
+    from quantization_amax_reduce_b200 import _check_padded_rows
+    _check_padded_rows([0, 300, 301, 430], [0, 320, 640], 960)       # fits
+    _check_padded_rows([0, 320, 320], [0, 960], 960)                  # empty at the end
+    with pytest.raises(ValueError, match="outside"):
+        _check_padded_rows([0, 300, 301, 430], [0, 320, 850], 960)    # 850 + 129 > 960
+    with pytest.raises(ValueError, match="outside"):
+        _check_padded_rows([0, 10], [-1], 960)
+    with pytest.raises(ValueError, match="one entry"):
+        _check_padded_rows([0, 10, 20], [0], 960)
+    with pytest.raises(ValueError, match="decrease"):
+        _check_padded_rows([0, 10, 5], [0, 320], 960)
