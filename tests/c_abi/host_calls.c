@@ -1,0 +1,72 @@
+/* A plain C99 consumer of libfp8attn: it includes only include/fp8attn.h and
+ * calls the entry points that do their work (or reject their arguments) on
+ * the host, so it runs without a GPU.  The selector examples are the ones the
+ * vLLM-Omni "Quantized KV Cache" page gives in its parameters table
+ * ("0,1,4-6" and "0-2,10"). */
+#include <stdio.h>
+#include <string.h>
+
+#include "fp8attn.h"
+
+static int fails = 0;
+#define CHECK(c)                                                        \
+  do {                                                                  \
+    if (!(c)) {                                                         \
+      printf("FAIL line %d: %s\n", __LINE__, #c);                       \
+      ++fails;                                                          \
+    }                                                                   \
+  } while (0)
+
+static int mask_is(const uint8_t* m, int n, const int* on, int n_on) {
+  int i, j;
+  for (i = 0; i < n; ++i) {
+    int want = 0;
+    for (j = 0; j < n_on; ++j)
+      if (on[j] == i) want = 1;
+    if ((m[i] != 0) != want) return 0;
+  }
+  return 1;
+}
+
+int main(void) {
+  uint8_t mask[12];
+  static const int sel_a[] = {0, 1, 4, 5, 6};
+  static const int sel_b[] = {0, 1, 2, 10};
+  fp8attn_ctx* ctx = (fp8attn_ctx*)0;
+
+  CHECK(fp8attn_ring_length() == 16);
+  CHECK(fp8attn_workspace_bytes(0) == 0);
+  CHECK(fp8attn_workspace_bytes(3) == 256 + 3 * 320);
+  CHECK(strcmp(fp8attn_status_string(FP8ATTN_OK), "ok") == 0);
+  CHECK(strcmp(fp8attn_status_string(12345), "unknown status") == 0);
+
+  CHECK(fp8attn_parse_selector("0,1,4-6", 12, mask) == FP8ATTN_OK);
+  CHECK(mask_is(mask, 12, sel_a, 5));
+  CHECK(fp8attn_parse_selector("0-2,10", 12, mask) == FP8ATTN_OK);
+  CHECK(mask_is(mask, 12, sel_b, 4));
+  CHECK(fp8attn_parse_selector((const char*)0, 12, mask) == FP8ATTN_OK);
+  CHECK(mask_is(mask, 12, sel_a, 0));
+  CHECK(fp8attn_parse_selector("6-4", 12, mask) != FP8ATTN_OK);
+  CHECK(fp8attn_parse_selector("12", 12, mask) != FP8ATTN_OK);
+
+  /* argument checks that return before any CUDA call */
+  CHECK(fp8attn_create(0, (void*)256, 1 << 20, (void*)0, &ctx) == FP8ATTN_ERR_INVALID);
+  CHECK(ctx == (fp8attn_ctx*)0);
+  CHECK(fp8attn_select_mode((const fp8attn_ctx*)0, (const uint8_t*)0, 0) == -1);
+  CHECK(fp8attn_regroup_heads((const void*)0, (void*)0, 0, 8, 2, 256, 1, (void*)0) ==
+        FP8ATTN_OK);
+  CHECK(fp8attn_regroup_heads((const void*)4096, (void*)(1 << 20), 4, 8, 3, 256, 1,
+                              (void*)0) == FP8ATTN_ERR_INVALID);
+  CHECK(fp8attn_varlen_fwd((const void*)0, (const void*)0, (const void*)0, (const int32_t*)16,
+                           1, 8, 0, 8, 128, (const float*)0, 0.0f, (void*)0, (int32_t*)0,
+                           (void*)0) == FP8ATTN_OK);
+  CHECK(fp8attn_varlen_fwd((const void*)16, (const void*)16, (const void*)16,
+                           (const int32_t*)16, 1, 8, 8, 8, 64, (const float*)16, 0.0f,
+                           (void*)16, (int32_t*)0, (void*)0) == FP8ATTN_ERR_UNSUPPORTED);
+
+  if (fails)
+    printf("FAILED (%d)\n", fails);
+  else
+    printf("ok\n");
+  return fails != 0;
+}

@@ -174,3 +174,22 @@ def test_padded_source_rows_checked_on_the_host():
         _check_padded_rows([0, 10, 20], [0], 960)
     with pytest.raises(ValueError, match="decrease"):
         _check_padded_rows([0, 10, 5], [0, 320], 960)
+
+
+def test_plain_c_consumer(tmp_path):
+    """The C ABI is usable from C99 with nothing but include/fp8attn.h and the
+    shared library: tests/c_abi/host_calls.c exercises the host-side entry
+    points and argument checks (no GPU needed)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler on this machine")
+    lib_dir = os.path.join(ROOT, "quantization_amax_reduce_b200")
+    exe = str(tmp_path / "host_calls")
+    subprocess.check_call([cc, "-std=c99", "-Wall", "-Wextra", "-Werror",
+                           "-I", os.path.join(ROOT, "include"),
+                           os.path.join(ROOT, "tests", "c_abi", "host_calls.c"),
+                           "-L", lib_dir, "-lfp8attn", f"-Wl,-rpath,{lib_dir}", "-o", exe])
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout + r.stderr
