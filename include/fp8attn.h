@@ -216,6 +216,34 @@ fp8attn_status fp8attn_varlen_fwd(const void* q8, const void* k8, const void* v8
                                   float softmax_scale, void* out, int32_t* d_error,
                                   void* stream);
 
+/* The rule that turns the softmax numerators into the E4M3 P operand of the
+ * PV product (the pages give none; both are defined in full here).  With
+ * c = ds_q ds_k softmax_scale log2(e), a per-row reference m (log2 units; the
+ * first 128-key block's max of s c, moved to a later block's max only when
+ * that exceeds m by more than 3) and t = s c - m + 5 <= 8:
+ *   FP8ATTN_P_LINEAR_LOG: code = RNE(8 t + 56) clamped to [0, 128] -- the
+ *     E4M3 bit pattern read as a fixed-point log2 (Mitchell's / Schraudolph's
+ *     piecewise-linear 2^t, exponent and mantissa filled linearly from t);
+ *     no exponential is evaluated.  NaN scores give code 0.  The row sum l
+ *     adds the E4M3 values of the codes.
+ *   FP8ATTN_P_EXP2: code = e4m3_rne(2^t) (2^t evaluated to about 2^-22
+ *     relative); l adds the unquantised 2^t.
+ * Both: out = (sum_j P_j v_j) ds_v / l, with P carried across moves of m by
+ * 2^(m_old - m_new). */
+typedef enum {
+  FP8ATTN_P_LINEAR_LOG = 0,
+  FP8ATTN_P_EXP2 = 1
+} fp8attn_p_rule;
+
+/* fp8attn_varlen_fwd with an explicit P rule (fp8attn_varlen_fwd uses
+ * FP8ATTN_P_EXP2).  Errors as fp8attn_varlen_fwd, and INVALID for an unknown
+ * rule. */
+fp8attn_status fp8attn_varlen_fwd_rule(const void* q8, const void* k8, const void* v8,
+                                       const int32_t* d_cu_seqlens, int batch, int max_seqlen,
+                                       int64_t total_tokens, int num_heads, int head_dim,
+                                       const float* d_descale_qkv, float softmax_scale,
+                                       int p_rule, void* out, int32_t* d_error, void* stream);
+
 /* Native-dtype attention for skipped layers (vLLM-Omni "Quantized KV Cache",
  * parameters table: selected layers keep the native dtype): the same
  * computation on bf16 q, k, v [T, num_heads, 128] with no quantisation. */
@@ -294,6 +322,17 @@ fp8attn_status fp8attn_regroup_heads(const void* d_src, void* d_dst, int64_t tok
  * FP8ATTN_ERR_CUDA on a CUDA error.  Takes about 1 s. */
 int fp8attn_selftest_bounded_waits(uint64_t mbar_limit_ns, int* h_gave_up, void* stream);
 
+/* Self-test of the score product (no counterpart in the pages; it checks
+ * the accumulation error that the tests' tie model assumes).  For each of
+ * `tiles` pairs of 128 x 128 E4M3 tiles -- rows [128 t, 128 t + 128) of
+ * d_q8 and d_k8, each [tiles * 128, 128] codes, 16-byte aligned -- writes
+ * S = Q K^T as fp32 to d_scores [tiles, 128, 128], computed with the FP8
+ * attention kernel's shared-memory layout, descriptors and MMA sequence.
+ * d_error: optional device int32 receiving FP8ATTN_ERR_TIMEOUT bits.
+ * Errors: INVALID (null pointers, tiles < 1, misaligned), CUDA. */
+fp8attn_status fp8attn_selftest_qk_scores(const void* d_q8, const void* d_k8, int64_t tiles,
+                                          float* d_scores, int32_t* d_error, void* stream);
+
 /* Allocation-free one-shot dynamic quantisation.  The pages have no
  * counterpart to this entry point; it exists for callers that cannot
  * allocate device memory -- for example an operator that an inference
@@ -319,7 +358,12 @@ int fp8attn_selftest_bounded_waits(uint64_t mbar_limit_ns, int* h_gave_up, void*
  * before any stream capture.  All calls share the one array, so calls whose
  * kernels overlap on the GPU (different streams, or concurrent graphs) race
  * and give wrong results: serialise them.  Device-side errors accumulate in
- * the array until read with fp8attn_quantize_qkv_noalloc_error().
+ * the array until read with fp8attn_quantize_qkv_noalloc_error().  After a
+ * device-side TIMEOUT the grid-barrier words may be left mid-count, so every
+ * later call on that device returns from its kernel at once, writing
+ * nothing, until fp8attn_quantize_qkv_noalloc_error() has reported the
+ * timeout and reset them.  The array belongs to the device current at the
+ * call (cudaGetDevice): make the inputs' device current before calling.
  * Returns an fp8attn_status. */
 int fp8attn_quantize_qkv_noalloc(const void* q, const void* k, const void* v, int64_t tok_stride,
                                  int64_t head_stride, const int32_t* d_src_seq_start,

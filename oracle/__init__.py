@@ -224,9 +224,12 @@ def _rows_arg(rows):
     return r, r.size
 
 
+P_LINEAR_LOG, P_EXP2 = "linear_log", "exp2"
+
+
 def attention_fp8(q8, k8, v8, cu, ds_qkv: Sequence[float], scale: Optional[float] = None,
                   pquant: bool = True, l_of_quantized: bool = False, rows=None,
-                  nthreads: int = 0, return_ambiguity: bool = False):
+                  nthreads: int = 0, return_ambiguity: bool = False, rule: str = P_EXP2):
     """fp64 attention on E4M3 codes [T, H, D]; returns [len(rows) or T, H, D].
 
     With ``pquant`` the PV product uses P quantised per block of 128 keys (in
@@ -235,6 +238,15 @@ def attention_fp8(q8, k8, v8, cu, ds_qkv: Sequence[float], scale: Optional[float
     r by more than 3 in log2 units; each block is carried exactly to the final
     max M; l is the sum of the unquantised exp(s - M) unless
     ``l_of_quantized``.
+
+    ``rule`` selects the quantisation of each block's P (both against the
+    same lagged reference r, t = (s - r) log2(e) + 5):
+    ``"exp2"``: code = e4m3(2^t) (RNE), l from the unquantised values as
+    above; ``"linear_log"``: code = 8 t + 56 rounded to the nearest integer
+    (ties to even) and clamped to [0, 128] -- the E4M3 bit pattern read as a
+    fixed-point log2, i.e. the piecewise-linear interpolation of 2^t between
+    powers of two rounded to the E4M3 grid -- with l the sum of the
+    quantised values and code 0 for NaN scores.
 
     With ``return_ambiguity`` also returns, per output, the largest change
     that P codes lying within an fp32 evaluation's error of a rounding tie
@@ -246,6 +258,8 @@ def attention_fp8(q8, k8, v8, cu, ds_qkv: Sequence[float], scale: Optional[float
     v8 = np.ascontiguousarray(v8, dtype=np.uint8)
     T, H, D = q8.shape
     cu = np.ascontiguousarray(np.asarray(cu, dtype=np.int32))
+    if rule not in (P_LINEAR_LOG, P_EXP2):
+        raise ValueError(f"unknown P rule {rule!r}")
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     r, nr = _rows_arg(rows)
@@ -254,7 +268,8 @@ def attention_fp8(q8, k8, v8, cu, ds_qkv: Sequence[float], scale: Optional[float
     amb = np.empty((n, H, D), dtype=np.float64) if return_ambiguity else None
     lib().or_attention_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(cu), cu.size - 1, H, D,
                            float(ds_qkv[0]), float(ds_qkv[1]), float(ds_qkv[2]),
-                           float(scale), int(bool(pquant)), int(bool(l_of_quantized)),
+                           float(scale), (2 if rule == P_LINEAR_LOG else 1) if pquant else 0,
+                           int(bool(l_of_quantized)),
                            _ptr(r), nr, _ptr(out), _ptr(amb), nthreads)
     return (out, amb) if return_ambiguity else out
 

@@ -117,6 +117,15 @@ uint8_t or_e4m3_encode(double y) {
     return (uint8_t)(sign | (efield << 3) | mant);
 }
 
+/* Decoded values of all 256 codes, filled from or_e4m3_value (only a
+ * lookup of the same function, so the attention loops do not re-decode). */
+static double dec_table[256];
+static pthread_once_t dec_once = PTHREAD_ONCE_INIT;
+static void fill_dec_table(void) {
+    int c;
+    for (c = 0; c < 256; ++c) dec_table[c] = or_e4m3_value((uint8_t)c);
+}
+
 /* Bulk encode of fp32 inputs (used by the exhaustive cast tests). */
 void or_e4m3_encode_f32_array(const float* y, int64_t n, uint8_t* out) {
     for (int64_t i = 0; i < n; ++i) out[i] = or_e4m3_encode((double)y[i]);
@@ -329,7 +338,8 @@ typedef struct {
     int B, H, D;
     double ds_q, ds_k, ds_v;
     double scale;             /* softmax scale (1/sqrt(D) by default) */
-    int pquant;               /* 0: p~ = p, 1: the block rule with a lagged reference max */
+    int pquant;               /* 0: p~ = p, 1: exp2 rule, 2: linear-log rule (both with the
+                                 block rule's lagged reference max) */
     int lrule;                /* 0: l = sum p, 1: l = sum p~ */
     const int64_t* rows;      /* token indices to evaluate (or NULL: all) */
     int64_t nrows;
@@ -341,7 +351,7 @@ typedef struct {
 
 static double elem(const att_job* j, const void* base, int64_t t, int h, int d) {
     int64_t idx = ((int64_t)t * j->H + h) * j->D + d;
-    if (j->kind == 0) return or_e4m3_value(((const uint8_t*)base)[idx]);
+    if (j->kind == 0) return dec_table[((const uint8_t*)base)[idx]];
     return (double)bf16_to_f32(((const uint16_t*)base)[idx]);
 }
 
@@ -357,55 +367,140 @@ static double elem(const att_job* j, const void* base, int64_t t, int h, int d) 
 #define OR_P_SCALE 32.0
 #define OR_P_LAG_LOG2 3.0
 
-/* Codes within reach of a rounding tie.  An implementation evaluates
- * y = 32 exp(s - r) in fp32 (exp2 of s*log2(e) - r*log2(e) + 5), so its y
- * carries a relative error of a few fp32 roundings of the exponent's terms
- * plus the exp2 approximation; bound it by
- *     eps(y) = 2^-20 * (2 + |s| log2(e) + |r| log2(e))
- * (16x the fp32 rounding of each term).  When [y(1-eps), y(1+eps)] holds a
- * tie between two E4M3 values, either code is a correct result of the rule;
- * the caller receives the largest output change such a flip can make. */
-static double code_ambiguity(double y, double s, double m) {
+/* Evaluation-error model of an implementation of the P rule, used only to
+ * tell which codes and which reference moves are decided at a tie (there
+ * either outcome is a correct result of the rule).  u = 2^-24 is the fp32
+ * unit roundoff.  The implementation evaluates, in log2 units,
+ *     t = s c + (5 - r2),   c = ds_q ds_k scale log2(e),   r2 = m c,
+ * where s is an fp32 accumulation of the 128 exact products of decoded
+ * codes, m the fp32 maximum of such scores over the reference block, c a
+ * product of three fp32 roundings of the scales and the fp32 value of
+ * log2(e), r2 and 5 - r2 one fp32 rounding each and t one fused
+ * multiply-add, then y = 2^t.  With A_j = scale ds_q ds_k sum_d |q_d k_jd|
+ * (so |s_j| <= A_j), A_r the largest A over the block that set r, and
+ * t* = (s - r) log2(e) + 5 the exact exponent:
+ *   - each score carries at most OR_ACC_ROUNDINGS u A of accumulation error
+ *     (in natural units; log2(e) times that in t);
+ *   - c is off by at most 4u relative, which reaches t through (s - r) c as
+ *     4u |t* - 5| (the same c multiplies s and m);
+ *   - the roundings of r2, of 5 - r2 and of the fused multiply-add add
+ *     u |r2|, u (5 + |r2|) and u |t|;
+ *   - 2^t itself is evaluated to within OR_EXP2_REL relative error.
+ * So y carries a relative error of at most
+ *     ln2 [log2(e) OR_ACC_ROUNDINGS u (A_j + A_r) + u (4|t* - 5| + 2|r2| + 5 + |t*|)]
+ *       + OR_EXP2_REL,
+ * doubled here for the second-order terms.  The reference move compares
+ * a = m_blk c with r2 + 3 (one fp32 rounding of the sum): a carries
+ * log2(e) OR_ACC_ROUNDINGS u A_blk + 5u |a|, r2 + 3 carries
+ * log2(e) OR_ACC_ROUNDINGS u A_r + 5u |r2| + u |r2 + 3|, doubled likewise.
+ * OR_ACC_ROUNDINGS bounds the tensor cores' fp32 accumulation of one
+ * 128-long dot product of E4M3 values (4 MMAs of 32 products): B200's
+ * error was measured at up to 7.9 u sum|q_d k_d| over 1.5 M random and
+ * adversarial scores (the GPU test of fp8attn_selftest_qk_scores checks
+ * the bound), so 16 leaves a factor of two.  OR_EXP2_REL bounds both exp2
+ * evaluations the kernel uses: the hardware approximation (measured at
+ * 1.45e-7 relative on [-10, 9]) and a degree-5 polynomial (2.13e-7, pinned
+ * by a CPU test). */
+#define OR_U 5.9604644775390625e-08   /* 2^-24 */
+#define OR_ACC_ROUNDINGS 16.0
+#define OR_EXP2_REL 4.76837158203125e-07   /* 2^-21 */
+
+static double p_rel_error(double t, double r2, double a_j, double a_r) {
     const double log2e = 1.4426950408889634;
-    double eps = ldexp(1.0, -20) * (2.0 + fabs(s) * log2e + fabs(m) * log2e);
+    double dt = log2e * OR_ACC_ROUNDINGS * OR_U * (a_j + a_r)
+              + OR_U * (4.0 * fabs(t - 5.0) + 2.0 * fabs(r2) + 5.0 + fabs(t));
+    return 2.0 * (0.6931471805599453 * dt + OR_EXP2_REL);
+}
+
+/* Largest change of p~ (in units of exp(r - M)) that a code decided at a
+ * tie can make: y = 32 exp(s - r) with relative error eps; 0 when
+ * y (1 - eps) and y (1 + eps) have the same code. */
+static double code_ambiguity(double y, double eps) {
     uint8_t lo = or_e4m3_encode(y * (1.0 - eps));
     uint8_t hi = or_e4m3_encode(y * (1.0 + eps));
     if (lo == hi) return 0.0;
     return fabs(or_e4m3_value(hi) - or_e4m3_value(lo)) / OR_P_SCALE;
 }
 
-/* Whether the reference max moves at a block is decided by an implementation
- * in fp32 (a block max of fp32 scores times the scale product, against r plus
- * the lag); when the fp64 comparison is within the same few fp32 roundings
- * of a tie, either decision is a correct result of the rule, and every later
- * P code of the row may differ.  Such rows are reported as unverifiable. */
-static int move_is_ambiguous(double blk_max, double r) {
+/* Whether a reference move (block max bm against reference r, natural
+ * units) is decided within the implementation's error of the threshold. */
+static int move_is_ambiguous(double bm, double a_blk, double r, double a_r) {
     const double log2e = 1.4426950408889634;
-    double a = blk_max * log2e, b = r * log2e + OR_P_LAG_LOG2;
-    double eps = ldexp(1.0, -18) * (4.0 + fabs(a));
-    return fabs(a - b) <= eps;
+    double a = bm * log2e, r2 = r * log2e, b = r2 + OR_P_LAG_LOG2;
+    double ea = log2e * OR_ACC_ROUNDINGS * OR_U * a_blk + 5.0 * OR_U * fabs(a);
+    double eb = log2e * OR_ACC_ROUNDINGS * OR_U * a_r + 5.0 * OR_U * fabs(r2) + OR_U * fabs(b);
+    return fabs(a - b) <= 2.0 * (ea + eb);
 }
 
-static void attend_one(const att_job* j, int64_t ri, int h, double* s_buf) {
+/* Linear-log P rule: the E4M3 code is 8 t + 56 rounded to the nearest
+ * integer (ties to even) and clamped to [0, 128], with t = (s - r) log2(e) + 5
+ * the exponent that the exp2 rule would raise 2 to.  In other words the
+ * E4M3 bit pattern is read as a fixed-point base-2 logarithm: the exponent
+ * field is the integer part of t, the mantissa field its fraction in
+ * eighths, so the value is the piecewise-linear interpolation of 2^t
+ * between powers of two (Mitchell's approximation) rounded to the E4M3
+ * grid.  A NaN score has code 0. */
+static uint8_t linear_log_code(double t) {
+    double y, n, frac;
+    if (isnan(t)) return 0;
+    y = 8.0 * t + 56.0;
+    if (y <= 0.0) return 0;
+    if (y >= 128.0) return 128;
+    n = floor(y);
+    frac = y - n;
+    if (frac > 0.5 || (frac == 0.5 && fmod(n, 2.0) == 1.0)) n += 1.0;
+    return (uint8_t)n;
+}
+
+/* The linear-log rule's implementation error in t (log2 units): the same
+ * score, scale and reference terms as p_rel_error, evaluated as
+ * y = sat(s c / 16 + (0.75 - r2 / 16)) = (8 t + 56) / 128: the roundings of
+ * r2, of 0.75 - r2/16 and of the fused multiply-add add u |r2|,
+ * u |12 - r2| and u |t + 7| (in t units), and no exponential is evaluated.
+ * Doubled for second-order terms.  A code is decided at a tie when 8 t + 56
+ * lies within 8 times this of a half-integer. */
+static double linear_log_t_error(double t, double r2, double a_j, double a_r) {
+    const double log2e = 1.4426950408889634;
+    double dt = log2e * OR_ACC_ROUNDINGS * OR_U * (a_j + a_r)
+              + OR_U * (4.0 * fabs(t - 5.0) + fabs(r2) + fabs(12.0 - r2) + fabs(t + 7.0));
+    return 2.0 * dt;
+}
+
+/* Largest change of p~ (in units of exp(r - M)) that a linear-log code
+ * decided at a tie can make. */
+static double linear_log_ambiguity(double t, double dt) {
+    uint8_t lo = linear_log_code(t - dt), hi = linear_log_code(t + dt);
+    if (lo == hi) return 0.0;
+    return fabs(or_e4m3_value(hi) - or_e4m3_value(lo)) / OR_P_SCALE;
+}
+
+static void attend_one(const att_job* j, int64_t ri, int h, double* s_buf, double* a_buf) {
     int64_t t = j->rows ? j->rows[ri] : ri;
     int b, d;
     int64_t k0, k1, kk;
-    double M = -INFINITY, l = 0.0, r = -INFINITY;
+    double M = -INFINITY, l = 0.0, r = -INFINITY, a_r = 0.0, amb_l = 0.0;
     int unverifiable = 0;
     double* o = j->out + (ri * j->H + h) * (int64_t)j->D;
     double* a = j->amb ? j->amb + (ri * j->H + h) * (int64_t)j->D : NULL;
     double dsq = j->kind == 0 ? j->ds_q : 1.0;
     double dsk = j->kind == 0 ? j->ds_k : 1.0;
     double dsv = j->kind == 0 ? j->ds_v : 1.0;
+    double sc = dsq * dsk * j->scale;
     for (b = 0; b < j->B; ++b)
         if (t >= j->cu[b] && t < j->cu[b + 1]) break;
     k0 = j->cu[b];
     k1 = j->cu[b + 1];
-    /* scores: dot of decoded values (exact in fp64 for E4M3), then scales */
+    /* scores: dot of decoded values (exact in fp64 for E4M3), then scales;
+     * A_j = the same sum of absolute products (the error model's scale) */
     for (kk = k0; kk < k1; ++kk) {
-        double acc = 0.0;
-        for (d = 0; d < j->D; ++d) acc += elem(j, j->q, t, h, d) * elem(j, j->k, kk, h, d);
-        s_buf[kk - k0] = acc * dsq * dsk * j->scale;
+        double acc = 0.0, aacc = 0.0;
+        for (d = 0; d < j->D; ++d) {
+            double pr = elem(j, j->q, t, h, d) * elem(j, j->k, kk, h, d);
+            acc += pr;
+            aacc += fabs(pr);
+        }
+        s_buf[kk - k0] = acc * sc;
+        a_buf[kk - k0] = aacc * fabs(sc);
         if (s_buf[kk - k0] > M) M = s_buf[kk - k0];
     }
     for (d = 0; d < j->D; ++d) o[d] = 0.0;
@@ -418,32 +513,61 @@ static void attend_one(const att_job* j, int64_t ri, int h, double* s_buf) {
         if ((kk - k0) % OR_P_BLOCK == 0) {
             /* entering a new block: its max, and whether the reference moves */
             int64_t e = kk + OR_P_BLOCK < k1 ? kk + OR_P_BLOCK : k1, x;
-            double bm = -INFINITY;
-            for (x = kk; x < e; ++x)
+            double bm = -INFINITY, a_blk = 0.0;
+            for (x = kk; x < e; ++x) {
                 if (s_buf[x - k0] > bm) bm = s_buf[x - k0];
+                if (a_buf[x - k0] > a_blk) a_blk = a_buf[x - k0];
+            }
             if (r == -INFINITY) {
                 r = bm;
+                a_r = a_blk;
             } else {
-                if (move_is_ambiguous(bm, r)) unverifiable = 1;
-                if (bm * 1.4426950408889634 > r * 1.4426950408889634 + OR_P_LAG_LOG2) r = bm;
+                if (move_is_ambiguous(bm, a_blk, r, a_r)) unverifiable = 1;
+                if (bm * 1.4426950408889634 > r * 1.4426950408889634 + OR_P_LAG_LOG2) {
+                    r = bm;
+                    a_r = a_blk;
+                }
             }
         }
-        if (j->pquant) {
+        if (j->pquant == 1) {
             double y = OR_P_SCALE * exp(s - r);
             pt = or_e4m3_value(or_e4m3_encode(y)) / OR_P_SCALE * exp(r - M);
             if (a) {
-                double amb = code_ambiguity(y, s, r) * exp(r - M);
+                double tt = (s - r) * 1.4426950408889634 + 5.0;
+                double eps = p_rel_error(tt, r * 1.4426950408889634, a_buf[kk - k0], a_r);
+                double amb = code_ambiguity(y, eps) * exp(r - M);
+                amb_l += amb;
+                if (amb > 0.0)
+                    for (d = 0; d < j->D; ++d) a[d] += amb * fabs(elem(j, j->v, kk, h, d));
+            }
+        } else if (j->pquant == 2) {
+            double tt = (s - r) * 1.4426950408889634 + 5.0;
+            pt = or_e4m3_value(linear_log_code(tt)) / OR_P_SCALE * exp(r - M);
+            if (a && !isnan(tt)) {
+                double dt = linear_log_t_error(tt, r * 1.4426950408889634, a_buf[kk - k0], a_r);
+                double amb = linear_log_ambiguity(tt, dt) * exp(r - M);
+                amb_l += amb;
                 if (amb > 0.0)
                     for (d = 0; d < j->D; ++d) a[d] += amb * fabs(elem(j, j->v, kk, h, d));
             }
         }
-        l += j->lrule ? pt : p;
+        l += (j->lrule || j->pquant == 2) ? pt : p;
         for (d = 0; d < j->D; ++d) o[d] += pt * elem(j, j->v, kk, h, d);
     }
-    for (d = 0; d < j->D; ++d) o[d] = o[d] * dsv / l;
-    if (a)
+    if (a && (j->lrule || j->pquant == 2)) {
+        /* l = sum p~ moves with the same codes: a flip by D changes the
+         * output by ds_v D (v_j - O/l) / (l + D), bounded by
+         * ds_v |D| (|v_j| + |O/l|) / (l - sum |D|) */
+        double lmin = l - amb_l;
         for (d = 0; d < j->D; ++d)
-            a[d] = (unverifiable && j->pquant) ? INFINITY : a[d] * dsv / l;
+            a[d] = (amb_l == 0.0) ? 0.0
+                 : (lmin > 0.0 ? (a[d] + amb_l * fabs(o[d] / l)) * dsv / lmin : INFINITY);
+    } else if (a) {
+        for (d = 0; d < j->D; ++d) a[d] = a[d] * dsv / l;
+    }
+    if (a && unverifiable && j->pquant)
+        for (d = 0; d < j->D; ++d) a[d] = INFINITY;
+    for (d = 0; d < j->D; ++d) o[d] = o[d] * dsv / l;
 }
 
 static void* att_worker(void* arg) {
@@ -453,14 +577,14 @@ static void* att_worker(void* arg) {
     double* s_buf;
     for (b = 0; b < j->B; ++b)
         if (j->cu[b + 1] - j->cu[b] > maxlen) maxlen = j->cu[b + 1] - j->cu[b];
-    s_buf = (double*)malloc(sizeof(double) * (size_t)(maxlen > 0 ? maxlen : 1));
+    s_buf = (double*)malloc(2 * sizeof(double) * (size_t)(maxlen > 0 ? maxlen : 1));
     for (;;) {
         int64_t w;
         pthread_mutex_lock(&j->lock);
         w = j->next++;
         pthread_mutex_unlock(&j->lock);
         if (w >= total) break;
-        attend_one(j, w / j->H, (int)(w % j->H), s_buf);
+        attend_one(j, w / j->H, (int)(w % j->H), s_buf, s_buf + (maxlen > 0 ? maxlen : 1));
     }
     free(s_buf);
     return NULL;
@@ -473,6 +597,7 @@ static int run_attention(att_job* j, int nthreads) {
     if (nthreads < 1) nthreads = 1;
     if (nthreads > 256) nthreads = 256;
     if (!j->rows) j->nrows = j->cu[j->B];
+    pthread_once(&dec_once, fill_dec_table);
     j->next = 0;
     pthread_mutex_init(&j->lock, NULL);
     for (i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, att_worker, j);

@@ -25,7 +25,7 @@ import numpy as np
 import torch
 
 __all__ = [
-    "DYNAMIC", "STATIC", "SKIP", "RING_LENGTH", "DEFAULT_MARGIN", "FP8AttnError", "lib",
+    "DYNAMIC", "STATIC", "SKIP", "P_LINEAR_LOG", "P_EXP2", "RING_LENGTH", "DEFAULT_MARGIN", "FP8AttnError", "lib",
     "Context", "varlen_fwd", "varlen_fwd_bf16", "parse_selector", "e4m3_encode",
     "launch_count", "load_scale_file", "save_scale_file", "read_error_word",
     "quantize_qkv_noalloc", "quantize_qkv_noalloc_error", "RING",
@@ -36,6 +36,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libfp8attn.so")
 
 DYNAMIC, STATIC, SKIP, RING = 0, 1, 2, 3
+P_LINEAR_LOG, P_EXP2 = 0, 1
 RING_LENGTH = 16
 DEFAULT_MARGIN = 1.5
 HEAD_DIM = 128
@@ -87,6 +88,7 @@ def lib() -> ctypes.CDLL:
         "fp8attn_set_ring_state": (I, [P, I, P, P, P]),
         "fp8attn_get_scales": (I, [P, I, P, P]),
         "fp8attn_varlen_fwd": (I, [P, P, P, P, I, I, I64, I, I, P, F, P, P, P]),
+        "fp8attn_varlen_fwd_rule": (I, [P, P, P, P, I, I, I64, I, I, P, F, I, P, P, P]),
         "fp8attn_varlen_fwd_bf16": (I, [P, P, P, P, I, I, I64, I, I, F, P, P, P]),
         "fp8attn_get_error": (I, [P, P]),
         "fp8attn_read_error_word": (I, [P, P]),
@@ -100,6 +102,7 @@ def lib() -> ctypes.CDLL:
         "fp8attn_quantize_qkv_noalloc_error": (I, [P]),
         "fp8attn_selftest_bounded_waits": (I, [ctypes.c_uint64, ctypes.POINTER(I), P]),
         "fp8attn_regroup_heads": (I, [P, P, I64, I, I, I, I, P]),
+        "fp8attn_selftest_qk_scores": (I, [P, P, I64, P, P, P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -404,10 +407,12 @@ def _attn_common(q, k, v, cu_seqlens, out, dtype):
 def varlen_fwd(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, cu_seqlens,
                max_seqlen: int, descale, softmax_scale: float = 0.0,
                out: Optional[torch.Tensor] = None, error: Optional[torch.Tensor] = None,
-               stream=None) -> torch.Tensor:
+               stream=None, p_rule: int = P_EXP2) -> torch.Tensor:
     """FP8 attention on packed E4M3 [T, H, 128] codes.  ``descale`` is a device
     pointer (int, e.g. ``Context.descale_ptr(layer)``) or a 3-element fp32 CUDA
-    tensor {ds_q, ds_k, ds_v}.  Returns bf16 [T, H, 128]."""
+    tensor {ds_q, ds_k, ds_v}.  ``p_rule`` picks how P is quantised for the PV
+    product (P_EXP2 or P_LINEAR_LOG, see fp8attn_p_rule in fp8attn.h).
+    Returns bf16 [T, H, 128]."""
     T, H, cu, out = _attn_common(q8, k8, v8, cu_seqlens, out, torch.uint8)
     if isinstance(descale, torch.Tensor):
         _require_cuda(descale, "descale")
@@ -416,11 +421,11 @@ def varlen_fwd(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, cu_seqlens,
         dptr = ctypes.c_void_p(descale.data_ptr())
     else:
         dptr = ctypes.c_void_p(int(descale))
-    _check(lib().fp8attn_varlen_fwd(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(cu), cu.numel() - 1,
-                                    int(max_seqlen), T, H, HEAD_DIM, dptr, float(softmax_scale),
-                                    _ptr(out), _ptr(error),
-                                    ctypes.c_void_p(_stream(stream, q8.device))),
-           "fp8attn_varlen_fwd")
+    _check(lib().fp8attn_varlen_fwd_rule(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(cu), cu.numel() - 1,
+                                         int(max_seqlen), T, H, HEAD_DIM, dptr,
+                                         float(softmax_scale), int(p_rule), _ptr(out),
+                                         _ptr(error), ctypes.c_void_p(_stream(stream, q8.device))),
+           "fp8attn_varlen_fwd_rule")
     return out
 
 
@@ -482,44 +487,24 @@ def quantize_qkv_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_s
     memory: every buffer, including the outputs ``q8``/``k8``/``v8`` and the
     3-float ``descale_out`` (and optional ``scale_out``), is the caller's, and
     the library keeps its reduction scratch in a fixed device array.  Calls
-    that overlap on the GPU race on that array."""
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        _require_cuda(t, name)
-        if t.dtype != torch.bfloat16:
-            raise ValueError(f"{name} must be bfloat16")
-    if q.stride() != k.stride() or q.stride() != v.stride() or q.shape[-1] != HEAD_DIM:
-        raise ValueError("q, k, v must share strides and have head_dim 128")
-    if q.shape != k.shape or q.shape != v.shape or q.stride(-1) != 1 or q.dim() not in (3, 4):
-        raise ValueError("q, k, v must be [T, H, 128] or [B, S_max, H, 128] with the channel "
-                         "contiguous")
-    if q.dim() == 4 and q.shape[0] > 1 and q.stride(0) != q.shape[1] * q.stride(1):
-        raise ValueError("a padded source needs its sequences back to back "
-                         "(stride(0) == S_max * stride(1))")
-    for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
-        _require_cuda(t, name)
-        if t.dtype != torch.uint8 or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous uint8 tensor")
-    _require_cuda(descale_out, "descale_out")
-    if descale_out.dtype != torch.float32 or descale_out.numel() < 3:
-        raise ValueError("descale_out must hold 3 fp32 values")
-    if scale_out is not None:
-        _require_cuda(scale_out, "scale_out")
-        if scale_out.dtype != torch.float32 or scale_out.numel() < 3:
-            raise ValueError("scale_out must hold 3 fp32 values")
-    H = q.shape[-2]
-    cu = _cu_tensor(cu_seqlens, q.device)
-    if total_tokens is None:
-        if src_seq_start is not None:
-            raise ValueError("total_tokens is required with a padded source")
-        total_tokens = q.shape[-3] if q.dim() == 3 else q.shape[0] * q.shape[1]
+    that overlap on the GPU race on that array.  Sources are checked as for
+    :meth:`Context.quantize_qkv`; the call runs with ``q``'s device current
+    (the library's array belongs to the current device)."""
+    H, tok_stride, head_stride, cu, B, total_tokens, sss = _qkv_source(
+        q, k, v, cu_seqlens, total_tokens, src_seq_start)
+    if cu.device != q.device or (sss is not None and sss.device != q.device):
+        raise ValueError(f"cu_seqlens and src_seq_start must be on {q.device}")
     for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
         _check_out(t, name, torch.uint8, int(total_tokens) * H * HEAD_DIM, q.device)
-    sss = None if src_seq_start is None else _cu_tensor(src_seq_start, q.device)
-    _check(lib().fp8attn_quantize_qkv_noalloc(
-        _ptr(q), _ptr(k), _ptr(v), q.stride(-3), q.stride(-2), _ptr(sss), _ptr(cu),
-        cu.numel() - 1, int(max_seqlen), int(total_tokens), H, HEAD_DIM, _ptr(q8), _ptr(k8),
-        _ptr(v8), _ptr(descale_out), _ptr(scale_out),
-        ctypes.c_void_p(_stream(stream, q.device))), "fp8attn_quantize_qkv_noalloc")
+    _check_out(descale_out, "descale_out", torch.float32, 3, q.device)
+    if scale_out is not None:
+        _check_out(scale_out, "scale_out", torch.float32, 3, q.device)
+    with torch.cuda.device(q.device):
+        _check(lib().fp8attn_quantize_qkv_noalloc(
+            _ptr(q), _ptr(k), _ptr(v), tok_stride, head_stride, _ptr(sss), _ptr(cu), B,
+            int(max_seqlen), int(total_tokens), H, HEAD_DIM, _ptr(q8), _ptr(k8), _ptr(v8),
+            _ptr(descale_out), _ptr(scale_out), ctypes.c_void_p(_stream(stream, q.device))),
+            "fp8attn_quantize_qkv_noalloc")
 
 
 def quantize_qkv_noalloc_error(stream=None) -> int:
@@ -569,6 +554,27 @@ def save_scale_file(path: str, layer_names: Sequence[str], values: np.ndarray) -
             for n, v in zip(layer_names, values)}
     with open(path, "w") as f:
         json.dump(data, f, indent=2)
+
+
+def selftest_qk_scores(q8: torch.Tensor, k8: torch.Tensor, stream=None) -> torch.Tensor:
+    """S = Q K^T for 128 x 128 tiles of E4M3 codes with the attention kernel's
+    MMA sequence: q8, k8 uint8 [tiles * 128, 128] on the device; returns fp32
+    [tiles, 128, 128] (a self-test of the tensor cores' accumulation)."""
+    for name, t in (("q8", q8), ("k8", k8)):
+        _require_cuda(t, name)
+        if t.dtype != torch.uint8 or not t.is_contiguous() or t.dim() != 2 or \
+                t.shape[1] != HEAD_DIM or t.shape[0] % 128 or t.shape[0] == 0:
+            raise ValueError(f"{name} must be a contiguous uint8 [tiles * 128, 128] tensor")
+    if q8.shape != k8.shape:
+        raise ValueError("q8 and k8 must have the same shape")
+    tiles = q8.shape[0] // 128
+    out = torch.empty((tiles, 128, 128), dtype=torch.float32, device=q8.device)
+    err = torch.zeros(1, dtype=torch.int32, device=q8.device)
+    _check(lib().fp8attn_selftest_qk_scores(_ptr(q8), _ptr(k8), tiles, _ptr(out), _ptr(err),
+                                            ctypes.c_void_p(_stream(stream, q8.device))),
+           "fp8attn_selftest_qk_scores")
+    _check(read_error_word(err, stream), "fp8attn_selftest_qk_scores (device)")
+    return out
 
 
 def selftest_bounded_waits(mbar_limit_ns: int = 50_000_000, device=None) -> int:

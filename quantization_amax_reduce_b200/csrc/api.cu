@@ -71,7 +71,8 @@ fp8attn_status check_attention(const void* q, const void* k, const void* v,
 fp8attn_status run_attention(const void* q, const void* k, const void* v, const int32_t* cu,
                              int batch, int max_seqlen, int64_t total_tokens, int num_heads,
                              int head_dim, const float* descale, float softmax_scale, void* out,
-                             int32_t* err, void* stream, int bf16) {
+                             int32_t* err, void* stream, int bf16, int p_rule) {
+  if (p_rule != FP8ATTN_P_LINEAR_LOG && p_rule != FP8ATTN_P_EXP2) return FP8ATTN_ERR_INVALID;
   fp8attn_status st = check_attention(q, k, v, cu, batch, max_seqlen, total_tokens, num_heads,
                                       head_dim, out);
   if (st != FP8ATTN_OK || total_tokens == 0) return st;
@@ -91,6 +92,7 @@ fp8attn_status run_attention(const void* q, const void* k, const void* v, const 
   a.out = out;
   a.err = err;
   a.bf16 = bf16;
+  a.p_rule = p_rule == FP8ATTN_P_EXP2 ? kPRuleExp2 : kPRuleLinearLog;
   const cudaError_t e = launch_attention(a, total_tokens, as_stream(stream));
   if (e != cudaSuccess) return FP8ATTN_ERR_CUDA;
   g_launches.fetch_add(1);
@@ -98,6 +100,8 @@ fp8attn_status run_attention(const void* q, const void* k, const void* v, const 
 }
 
 }  // namespace
+
+void fp8attn::note_launch() { g_launches.fetch_add(1); }
 
 extern "C" {
 
@@ -372,7 +376,30 @@ fp8attn_status fp8attn_varlen_fwd(const void* q8, const void* k8, const void* v8
                                   const float* d_descale_qkv, float softmax_scale, void* out,
                                   int32_t* d_error, void* stream) {
   return run_attention(q8, k8, v8, d_cu_seqlens, batch, max_seqlen, total_tokens, num_heads,
-                       head_dim, d_descale_qkv, softmax_scale, out, d_error, stream, 0);
+                       head_dim, d_descale_qkv, softmax_scale, out, d_error, stream, 0,
+                       FP8ATTN_P_EXP2);
+}
+
+fp8attn_status fp8attn_varlen_fwd_rule(const void* q8, const void* k8, const void* v8,
+                                       const int32_t* d_cu_seqlens, int batch, int max_seqlen,
+                                       int64_t total_tokens, int num_heads, int head_dim,
+                                       const float* d_descale_qkv, float softmax_scale,
+                                       int p_rule, void* out, int32_t* d_error, void* stream) {
+  return run_attention(q8, k8, v8, d_cu_seqlens, batch, max_seqlen, total_tokens, num_heads,
+                       head_dim, d_descale_qkv, softmax_scale, out, d_error, stream, 0, p_rule);
+}
+
+fp8attn_status fp8attn_selftest_qk_scores(const void* d_q8, const void* d_k8, int64_t tiles,
+                                          float* d_scores, int32_t* d_error, void* stream) {
+  if (!d_q8 || !d_k8 || !d_scores || tiles < 1 || tiles > 0x7FFFFFFF / 128)
+    return FP8ATTN_ERR_INVALID;
+  if (!aligned(d_q8, 16) || !aligned(d_k8, 16) || !aligned(d_scores, 16))
+    return FP8ATTN_ERR_INVALID;
+  if (launch_qk_scores_probe(d_q8, d_k8, tiles, d_scores, d_error, as_stream(stream)) !=
+      cudaSuccess)
+    return FP8ATTN_ERR_CUDA;
+  g_launches.fetch_add(1);
+  return FP8ATTN_OK;
 }
 
 fp8attn_status fp8attn_varlen_fwd_bf16(const void* q, const void* k, const void* v,
@@ -381,7 +408,8 @@ fp8attn_status fp8attn_varlen_fwd_bf16(const void* q, const void* k, const void*
                                        float softmax_scale, void* out, int32_t* d_error,
                                        void* stream) {
   return run_attention(q, k, v, d_cu_seqlens, batch, max_seqlen, total_tokens, num_heads,
-                       head_dim, nullptr, softmax_scale, out, d_error, stream, 1);
+                       head_dim, nullptr, softmax_scale, out, d_error, stream, 1,
+                       FP8ATTN_P_EXP2);
 }
 
 fp8attn_status fp8attn_get_error(fp8attn_ctx* ctx, void* stream) {

@@ -98,6 +98,21 @@ __device__ __forceinline__ void note_error(AttnParams& p, Bars& bars, uint32_t b
   if (p.err) atomicOr(reinterpret_cast<unsigned int*>(p.err), bit);
 }
 
+// Keys past the end of a sequence share the last K/V tile with the next
+// sequence's first rows (or TMA zero fill past the tensor).  Their scores are
+// masked to -inf, so P is 0 there, but 0 * NaN (or Inf) in the PV product is
+// NaN: the rows of V at or after `valid` are zeroed in shared memory before
+// the PV MMA reads them.  A row is 128 bytes of every 128B-swizzled tile (the
+// swizzle permutes 16-byte chunks within a row), so the rows form one
+// contiguous range.  Called by all 32 lanes of the MMA warp.
+__device__ __forceinline__ void zero_tail_rows(uint8_t* tile, int valid, int lane) {
+  uint4* p = reinterpret_cast<uint4*>(tile + valid * 128);
+  const int n = (128 - valid) * 8;
+  for (int i = lane; i < n; i += 32) p[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async();   // generic-proxy stores -> tensor-core operand reads
+  __syncwarp();
+}
+
 __global__ void __launch_bounds__(kThreadsAttn, 1)
 attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, AttnParams p) {
@@ -263,8 +278,13 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       for (int j = 0; j < nkv && ok; ++j) {
         const int st = j % C::kStages;
         const int st1 = (j + 1) % C::kStages;
-        ok = mbar_wait(&bars.v_full[st], (j / C::kStages) & 1, abort_flag) &&
-             mbar_wait(&bars.p_full[0], j & 1, abort_flag);
+        ok = mbar_wait(&bars.v_full[st], (j / C::kStages) & 1, abort_flag);
+        if (ok && j + 1 == nkv && (len & 127)) {
+          // both 64-column halves of the last, partial V tile
+          zero_tail_rows(sv + st * C::kTile, len & 127, lane);
+          zero_tail_rows(sv + st * C::kTile + 16384, len & 127, lane);
+        }
+        ok = ok && mbar_wait(&bars.p_full[0], j & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
         issue_pv(0, st, j);
@@ -474,6 +494,7 @@ struct Fp8Barriers {
   int abort_flag;
 };
 
+template <int kRule>
 __global__ void __launch_bounds__(kThreadsAttn, 1)
 attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -637,6 +658,7 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (!ok) break;
       }
       ok = mbar_wait(&bars.v_full[st], (j / C::kStages) & 1, abort_flag);
+      if (ok && j + 1 == nkv && (len & 127)) zero_tail_rows(sv + st * C::kTile, len & 127, lane);
       for (int i = 0; i < 2 && ok; ++i) {
         ok = mbar_wait(&bars.p_full[i][j & 1], (j >> 1) & 1, abort_flag);
         if (!ok) break;
@@ -697,28 +719,65 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
       const float m_blk = mx * cscale;
       const bool moved = m_blk > m_run + kRefLag;
       const float m_new = moved ? m_blk : m_run;
-      const float neg = kPOffsetLog2 - m_new;
-      const uint64_t c2 = f2_pack(cscale, cscale);
-      const uint64_t n2 = f2_pack(neg, neg);
-      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
       uint32_t pw[32];
+      float sum;
+      if (kRule == kPRuleExp2) {
+        const float neg = kPOffsetLog2 - m_new;
+        const uint64_t c2 = f2_pack(cscale, cscale);
+        const uint64_t n2 = f2_pack(neg, neg);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int k = 0; k < 64; ++k) {
-        const uint64_t t = f2_fma(f2_pack(__uint_as_float(u[2 * k]), __uint_as_float(u[2 * k + 1])),
-                                  c2, n2);
-        float t0, t1;
-        f2_unpack(t, t0, t1);
-        uint64_t e;
-        if (k % kPolyEvery == kPolyEvery - 1)
-          e = f2_exp2_poly(f2_pack(fmaxf(t0, -126.0f), fmaxf(t1, -126.0f)));
-        else
-          e = f2_pack(ex2_approx(t0), ex2_approx(t1));
-        acc[k & 3] = f2_add(acc[k & 3], e);
-        float e0, e1;
-        f2_unpack(e, e0, e1);
-        const uint32_t hh = cvt_e4m3x2(e0, e1);
-        if (k & 1) pw[k >> 1] |= hh << 16;
-        else pw[k >> 1] = hh;
+        for (int k = 0; k < 64; ++k) {
+          const uint64_t t = f2_fma(f2_pack(__uint_as_float(u[2 * k]), __uint_as_float(u[2 * k + 1])),
+                                    c2, n2);
+          float t0, t1;
+          f2_unpack(t, t0, t1);
+          uint64_t e;
+          if (k % kPolyEvery == kPolyEvery - 1)
+            e = f2_exp2_poly(f2_pack(fmaxf(t0, -126.0f), fmaxf(t1, -126.0f)));
+          else
+            e = f2_pack(ex2_approx(t0), ex2_approx(t1));
+          acc[k & 3] = f2_add(acc[k & 3], e);
+          float e0, e1;
+          f2_unpack(e, e0, e1);
+          const uint32_t hh = cvt_e4m3x2(e0, e1);
+          if (k & 1) pw[k >> 1] |= hh << 16;
+          else pw[k >> 1] = hh;
+        }
+        float a0, a1;
+        f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
+        sum = a0 + a1;
+      } else {
+        // Linear-log rule: code = RNE(8 t + 56) clamped to [0, 128], with
+        // t = s c - m + 5, i.e. the E4M3 bit pattern read as a fixed-point
+        // log2 (exponent and mantissa filled linearly from t).  Computed as
+        // y = sat(s c/16 + (0.75 - m/16)) = (8 t + 56) / 128 in [0, 1] (one
+        // rounding; NaN and -inf scores give 0), then y + 1.5 * 2^16 rounds
+        // 128 y to an integer in the low mantissa bits.  l sums the E4M3
+        // values of the codes (pairs summed exactly in f16 first where
+        // representable, then in fp32).
+        const float a16 = cscale * 0.0625f;
+        const float b16 = 0.75f - m_new * 0.0625f;
+        const uint64_t magic2 = f2_pack(98304.0f, 98304.0f);   // 1.5 * 2^16
+        float lacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        uint32_t hprev = 0;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const float y0 = fma_sat(__uint_as_float(u[4 * k + 0]), a16, b16);
+          const float y1 = fma_sat(__uint_as_float(u[4 * k + 1]), a16, b16);
+          const float y2 = fma_sat(__uint_as_float(u[4 * k + 2]), a16, b16);
+          const float y3 = fma_sat(__uint_as_float(u[4 * k + 3]), a16, b16);
+          uint32_t ra, rb, rc, rd;
+          asm("mov.b64 {%0, %1}, %2;" : "=r"(ra), "=r"(rb) : "l"(f2_add(f2_pack(y0, y1), magic2)));
+          asm("mov.b64 {%0, %1}, %2;" : "=r"(rc), "=r"(rd) : "l"(f2_add(f2_pack(y2, y3), magic2)));
+          const uint32_t c01 = prmt(ra, rb, 0x0040u);   // code0 | code1 << 8
+          const uint32_t c23 = prmt(rc, rd, 0x0040u);
+          pw[k] = prmt(c01, c23, 0x5410u);
+          const uint32_t h = hadd2(cvt_f16x2_from_e4m3x2(c01), cvt_f16x2_from_e4m3x2(c23));
+          if (k & 1) lacc[(k >> 1) & 3] = add_f16x2_to_f32(lacc[(k >> 1) & 3], hadd2(hprev, h));
+          else hprev = h;
+        }
+        sum = (lacc[0] + lacc[1]) + (lacc[2] + lacc[3]);
       }
       // P row -> shared memory (buffer j % 2 is free: S_i(j) complete means
       // PV_i(j-2), its last reader, is done)
@@ -728,12 +787,6 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
             make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
       fence_proxy_async();
-      float sum;
-      {
-        float a0, a1;
-        f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
-        sum = a0 + a1;
-      }
       const float alpha = ex2_approx(m_run - m_new);   // 0 on the first block, 1 unless moved
       l_run = l_run * alpha + sum;
       if (j > 0 && __any_sync(0xFFFFFFFFu, moved)) {
@@ -805,6 +858,79 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
   if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
+// ---------------------------------------------------------------------------
+// Self-test of the score product: S = Q K^T for 128 x 128 tiles of E4M3
+// codes, computed with the attention kernel's operand layout, descriptors
+// and MMA sequence (4 x K=32), written out in fp32 so that the tensor cores'
+// accumulation error can be checked against exact scores.
+// ---------------------------------------------------------------------------
+
+struct ProbeSmem {
+  uint8_t q[128 * 128];
+  uint8_t k[128 * 128];
+  uint64_t tma_bar, mma_bar;
+  uint32_t tmem_base;
+};
+
+__global__ void __launch_bounds__(128, 1)
+qk_scores_probe_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_k, float* scores, int32_t* err) {
+  extern __shared__ uint8_t smem_raw[];
+  ProbeSmem& sm = *reinterpret_cast<ProbeSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.tma_bar, 1);
+    mbar_init(&sm.mma_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&sm.tmem_base, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  if (threadIdx.x == 0) {
+    mbar_expect_tx(&sm.tma_bar, 2 * 16384);
+    tma_load_3d(sm.q, &tm_q, &sm.tma_bar, 0, 0, 128 * blockIdx.x);
+    tma_load_3d(sm.k, &tm_k, &sm.tma_bar, 0, 0, 128 * blockIdx.x);
+  }
+  bool ok = mbar_wait(&sm.tma_bar, 0, nullptr);
+  if (warp == 0 && ok) {
+    tc_fence_after();
+    const uint32_t id_qk = make_idesc(0, 0, 128, 0);
+    const uint64_t dq = make_sdesc_sw128(smem_u32(sm.q), 16, 1024);
+    const uint64_t dk = make_sdesc_sw128(smem_u32(sm.k), 16, 1024);
+    if (elect_one()) {
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tmem, dq + 2 * kk, dk + 2 * kk, id_qk, kk > 0);
+      mma_commit(&sm.mma_bar);
+    }
+    __syncwarp();
+  }
+  ok = ok && mbar_wait(&sm.mma_bar, 0, nullptr);
+  if (!ok && threadIdx.x == 0 && err) atomicOr(reinterpret_cast<unsigned int*>(err), kErrTimeout);
+  if (ok) {
+    tc_fence_after();
+    const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
+    float* row = scores + (static_cast<int64_t>(blockIdx.x) * 128 + threadIdx.x) * 128;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_off + 32 * c, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int x = 0; x < 32; ++x) row[32 * c + x] = __uint_as_float(r[x]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -841,19 +967,19 @@ bool make_qkv_map(CUtensorMap* m, const void* base, int64_t T, int H, bool bf16)
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool kFp8>
+template <bool kFp8, int kRule>
 cudaError_t launch_attention_t(const AttnLaunch& a, int64_t T, cudaStream_t stream) {
   CUtensorMap mq, mk, mv;
   if (!make_qkv_map(&mq, a.q, T, a.heads, !kFp8) || !make_qkv_map(&mk, a.k, T, a.heads, !kFp8) ||
       !make_qkv_map(&mv, a.v, T, a.heads, !kFp8))
     return cudaErrorInvalidValue;
   // FP8 runs the P-in-shared-memory kernel; BF16 keeps P in TMEM
-  auto kernel = kFp8 ? attn_fwd_fp8_kernel : attn_fwd_bf16_kernel;
+  auto kernel = kFp8 ? attn_fwd_fp8_kernel<kRule> : attn_fwd_bf16_kernel;
   const int smem_bytes = kFp8 ? Fp8Cfg::kSmemBytes : Bf16Cfg::kSmemBytes;
   // the shared-memory opt-in is a per-device function attribute: set it once
   // for each device this process launches on
   static std::mutex mu;
-  static uint64_t attr_set = 0;   // bit d: done on device d
+  static uint64_t attr_set = 0;   // bit d: done on device d (one per instantiation)
   {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -886,9 +1012,24 @@ cudaError_t launch_attention_t(const AttnLaunch& a, int64_t T, cudaStream_t stre
 
 }  // namespace
 
+cudaError_t launch_qk_scores_probe(const void* q8, const void* k8, int64_t tiles, float* scores,
+                                   int32_t* err, cudaStream_t stream) {
+  CUtensorMap mq, mk;
+  if (!make_qkv_map(&mq, q8, tiles * 128, 1, false) || !make_qkv_map(&mk, k8, tiles * 128, 1, false))
+    return cudaErrorInvalidValue;
+  const int smem_bytes = static_cast<int>(sizeof(ProbeSmem)) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(qk_scores_probe_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  if (e != cudaSuccess) return e;
+  qk_scores_probe_kernel<<<static_cast<unsigned>(tiles), 128, smem_bytes, stream>>>(mq, mk, scores,
+                                                                                 err);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_attention(const AttnLaunch& a, int64_t total_tokens, cudaStream_t stream) {
-  if (a.bf16) return launch_attention_t<false>(a, total_tokens, stream);
-  return launch_attention_t<true>(a, total_tokens, stream);
+  if (a.bf16) return launch_attention_t<false, kPRuleExp2>(a, total_tokens, stream);
+  if (a.p_rule == kPRuleExp2) return launch_attention_t<true, kPRuleExp2>(a, total_tokens, stream);
+  return launch_attention_t<true, kPRuleLinearLog>(a, total_tokens, stream);
 }
 
 }  // namespace fp8attn

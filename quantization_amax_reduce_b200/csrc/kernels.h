@@ -45,9 +45,22 @@ struct AttnLaunch {
   void* out;                     // bf16 [T, H, 128]
   int32_t* err;                  // device error word or null
   int bf16;                      // 1 = native bf16 inputs (skip-layer path)
+  int p_rule;                    // FP8 only: kPRuleLinearLog or kPRuleExp2
 };
 
+// P rules of the FP8 kernel (the values of fp8attn_p_rule in fp8attn.h).
+constexpr int kPRuleLinearLog = 0;
+constexpr int kPRuleExp2 = 1;
+
 cudaError_t launch_attention(const AttnLaunch& p, int64_t total_tokens, cudaStream_t stream);
+
+// S = Q K^T for `tiles` 128 x 128 tiles of E4M3 codes ([tiles * 128, 128]
+// each), with the FP8 attention kernel's MMA sequence; fp32 [tiles, 128, 128].
+cudaError_t launch_qk_scores_probe(const void* q8, const void* k8, int64_t tiles, float* scores,
+                                   int32_t* err, cudaStream_t stream);
+
+// Counts one successful kernel launch (fp8attn_launch_count).
+void note_launch();
 
 // [T, H, hb] <-> [G, T, H/G, hb] (to_groups = 1 / 0); hb a multiple of 16,
 // H a multiple of G, 16-byte aligned, non-overlapping buffers.

@@ -522,6 +522,10 @@ __global__ void __launch_bounds__(kThreads) quant_noalloc_kernel(NoAllocArgs n) 
   __shared__ float s_scale[2][3];
   const QuantArgs& a = n.a;
   uint32_t* scratch = n.scratch;
+  // A call that timed out may have left the barrier words mid-count: until
+  // fp8attn_quantize_qkv_noalloc_error has reported the timeout and reset
+  // them, every call leaves at once (outputs untouched).
+  if (*reinterpret_cast<volatile uint32_t*>(scratch + kNoAllocWordErr) & kErrTimeout) return;
   if (!seqlens_ok(a)) {
     if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(scratch + kNoAllocWordErr, kErrSeqlens);
     return;
@@ -719,6 +723,7 @@ int fp8attn_quantize_qkv_noalloc(const void* q, const void* k, const void* v, in
   const void* fn = contig ? reinterpret_cast<const void*>(&quant_noalloc_kernel<true>)
                           : reinterpret_cast<const void*>(&quant_noalloc_kernel<false>);
   if (cudaLaunchKernelExC(&cfg, fn, args) != cudaSuccess) return 2;
+  note_launch();
   return 0;
 }
 

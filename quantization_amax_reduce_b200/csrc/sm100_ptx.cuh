@@ -295,6 +295,44 @@ __device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
   return r;
 }
 
+// a * b + c, one rounding, clamped to [0, 1] (NaN gives +0).
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float d;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Byte permute: result byte i = byte (sel >> 4i) & 7 of {b, a} (a = bytes 0-3).
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// The two E4M3 codes in the low 16 bits of `x` -> their exact f16 values
+// (low code -> low half).
+__device__ __forceinline__ uint32_t cvt_f16x2_from_e4m3x2(uint32_t x) {
+  uint32_t d;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, lo;\n\t}" : "=r"(d) : "r"(x));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t hadd2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// acc + (low f16 of h) + (high f16 of h), each add in fp32 (mixed precision).
+__device__ __forceinline__ float add_f16x2_to_f32(float acc, uint32_t h) {
+  float d;
+  asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\t"
+      "add.rn.f32.f16 %0, lo, %2;\n\tadd.rn.f32.f16 %0, hi, %0;\n\t}"
+      : "=f"(d) : "r"(h), "f"(acc));
+  return d;
+}
+
 // ---------------------------------------------------------------------------
 // Packed fp32 pairs (sm_100 f32x2 arithmetic) and 3-input max
 // ---------------------------------------------------------------------------
@@ -337,7 +375,7 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // (callers clamp from below).  Cody-Waite style reduction x = j + f with j
 // = nearest integer (1.5 * 2^23 added and removed), f in [-1/2, 1/2]; 2^f
 // from a degree-5 polynomial fitted here by the Remez exchange algorithm
-// for minimum relative error (2.1e-7 evaluated in fp32); the integer j
+// for minimum relative error (2.13e-7 evaluated in fp32); the integer j
 // goes straight into the exponent bits.
 __device__ __forceinline__ uint64_t f2_exp2_poly(uint64_t x) {
   const uint64_t kShift = f2_pack(12582912.0f, 12582912.0f);        // 1.5 * 2^23

@@ -3,7 +3,7 @@ C-ABI binding, run the oracle on the same seeded inputs, compare."""
 from __future__ import annotations
 
 import math
-from typing import Optional, Sequence
+from typing import Optional, Sequence, Tuple
 
 import numpy as np
 import torch
@@ -11,13 +11,23 @@ import torch
 import oracle
 import synthetic
 
-# Attention tolerance against the oracle (fp64 with the same P rule):
-# max err <= 1e-2 and mean err <= 1e-3, with err = |got - ref| / max(1, |ref|).
-# For outputs of magnitude <= 1 this is the absolute error; above 1 it is
-# relative, because a bf16 output cannot hold a value of magnitude >= 4 to
-# within 1e-2 (half a bf16 ulp there is 1/64).
+# Attention tolerance against the oracle (fp64, same P rule): max abs error
+# <= 1e-2 and mean abs error <= 1e-3.  Each output's error is the absolute
+# difference less two allowances that no correct implementation can avoid:
+# the oracle's tie allowance (P codes within the kernel's evaluation error of
+# an E4M3 rounding tie, where either code is a correct result of the rule)
+# and half a bf16 ulp of the output (the kernel's result is a bf16 value:
+# RNE to bf16 moves it by up to half the spacing of bf16 numbers there).
 MAX_ABS_TOL = 1e-2
 MEAN_ABS_TOL = 1e-3
+# Outputs of rows whose reference-max move was decided within the kernel's
+# evaluation error of the threshold cannot be compared; more than this
+# fraction of them would hide a wrong rule.
+MAX_EXCLUDED_FRACTION = 1e-3
+
+# Per-check records, printed as one table at the end of the session
+# (tests/conftest.py), so they reach the log even when every check passes.
+RECORDS = []
 
 
 class OracleLayer:
@@ -87,21 +97,37 @@ def sample_rows(cu: np.ndarray, per_seq: int, seed: int = 0) -> np.ndarray:
         n = s1 - s0
         if n == 0:
             continue
+        # the first two query tiles' edges, every row of the last query block's
+        # tile starts and ends (the ragged tail), and the middle
         pick = {0, n - 1, min(127, n - 1), min(128, n - 1), min(255, n - 1), min(256, n - 1),
-                (n - 1) // 128 * 128, n // 2}
+                (n - 1) // 128 * 128, max(0, (n - 1) // 128 * 128 - 1), (n - 1) // 256 * 256,
+                max(0, n - 129), n // 2}
         k = max(0, min(per_seq, n) - len(pick))
         pick.update(rng.choice(n, size=min(k, n), replace=False).tolist())
         rows.extend(s0 + r for r in sorted(pick))
     return np.array(sorted(set(rows)), dtype=np.int64)
 
 
-def attention_errors(got: torch.Tensor, want, rows: Optional[np.ndarray] = None):
-    """(max, mean) of |got - ref| / max(1, |ref|).  `want` is the oracle output
-    or an (output, ambiguity) pair; the ambiguity allowance (P codes within an
-    fp32 evaluation's error of a rounding tie, where either neighbouring code
-    is a correct result of the rule) is subtracted first, and outputs with an
-    infinite allowance (a row whose reference-max move was decided at the
-    threshold) are left out."""
+def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
+    """Half the spacing of bf16 numbers at |x| (bf16 keeps 8 significant
+    bits: spacing 2^(e-7) in [2^e, 2^(e+1)); subnormal spacing below 2^-126)."""
+    a = np.maximum(np.abs(np.asarray(x, dtype=np.float64)), 2.0 ** -126)
+    e = np.floor(np.log2(a))
+    return np.ldexp(1.0, (e - 8).astype(np.int64))
+
+
+def attention_errors(got: torch.Tensor, want, rows: Optional[np.ndarray] = None) -> dict:
+    """Error statistics of a bf16 attention output against the oracle.
+
+    ``want`` is the oracle's fp64 output or an (output, allowance) pair.
+    Outputs where the oracle is not finite (a NaN or Inf input in the
+    sequence's own Q/K/V) must be non-finite in ``got`` too and are not part
+    of the statistics.  Returned keys: ``max``/``mean`` of the gated error
+    max(0, |got - ref| - allowance - bf16_half_ulp), ``plain_max``/
+    ``plain_mean`` of |got - ref| over the same outputs, ``n`` outputs
+    compared, ``n_tie`` with a tie allowance, ``n_excluded`` in rows decided
+    at the threshold, ``n_nonfinite_ok`` non-finite outputs that matched the
+    oracle's, ``n_nonfinite_bad`` that did not, ``max_ref``."""
     amb = np.zeros(1)
     if isinstance(want, tuple):
         want, amb = want
@@ -109,25 +135,54 @@ def attention_errors(got: torch.Tensor, want, rows: Optional[np.ndarray] = None)
     if rows is not None:
         g = g[rows]
     amb = np.broadcast_to(amb, want.shape)
-    keep = np.isfinite(amb)
-    if not keep.any():
-        return 0.0, 0.0
-    d = np.maximum(np.abs(g - want)[keep] - amb[keep], 0.0) / np.maximum(1.0, np.abs(want[keep]))
-    return float(d.max()), float(d.mean())
+    ref_finite = np.isfinite(want)
+    n_nf_bad = int(np.sum(~ref_finite & np.isfinite(g)) + np.sum(ref_finite & ~np.isfinite(g)))
+    n_nf_ok = int(np.sum(~ref_finite & ~np.isfinite(g)))
+    excluded = ref_finite & ~np.isfinite(amb)
+    keep = ref_finite & np.isfinite(amb) & np.isfinite(g)
+    st = dict(n=int(keep.sum()), n_tie=int(((amb > 0) & keep).sum()),
+              n_excluded=int(excluded.sum()), n_nonfinite_ok=n_nf_ok,
+              n_nonfinite_bad=n_nf_bad, max=0.0, mean=0.0, plain_max=0.0, plain_mean=0.0,
+              max_ref=float(np.abs(want[ref_finite]).max()) if ref_finite.any() else 0.0)
+    if keep.any():
+        gk, wk, ak = g[keep], want[keep], amb[keep]
+        plain = np.abs(gk - wk)
+        gated = np.maximum(plain - ak - bf16_half_ulp(np.maximum(np.abs(wk), np.abs(gk))), 0.0)
+        st.update(max=float(gated.max()), mean=float(gated.mean()),
+                  plain_max=float(plain.max()), plain_mean=float(plain.mean()))
+    return st
 
 
-def assert_attention_close(got, want, rows=None, what="attention"):
-    g = got.float().cpu().numpy()
+def unquantized_errors(got: torch.Tensor, ref: np.ndarray, rows=None) -> Tuple[float, float]:
+    """(max, mean) of |got - ref| against fp64 attention on the unquantised
+    bf16 inputs: reported beside the parity figures, not gated."""
+    g = got.float().cpu().numpy().astype(np.float64)
     if rows is not None:
         g = g[rows]
-    assert np.isfinite(g).all(), f"{what}: non-finite output"
-    mx, mean = attention_errors(got, want, rows)
-    ref = want[0] if isinstance(want, tuple) else want
-    n_amb = int((want[1] > 0).sum()) if isinstance(want, tuple) else 0
-    n_out = int(np.isinf(want[1]).sum()) if isinstance(want, tuple) else 0
-    print(f"{what}: max|err| {mx:.3e} mean|err| {mean:.3e} (max|ref| {np.abs(ref).max():.3e}, "
-          f"{n_amb} outputs with a tie allowance, {n_out} in rows decided at the threshold)")
-    assert mx <= MAX_ABS_TOL and mean <= MEAN_ABS_TOL, (what, mx, mean)
-    # threshold ties are rare; many of them would hide a wrong reference rule
-    assert n_out <= max(2 * ref.shape[-1], ref.size // 100), (what, n_out)
-    return mx, mean
+    d = np.abs(g - ref)
+    d = d[np.isfinite(d)]
+    return (float(d.max()), float(d.mean())) if d.size else (0.0, 0.0)
+
+
+def assert_attention_close(got, want, rows=None, what="attention", unquantized=None):
+    """Gate: gated max <= 1e-2, gated mean <= 1e-3, non-finite outputs where
+    and only where the oracle's are, excluded outputs <= 0.1 %.  The figures
+    go into the failure message and into the session summary.  With
+    ``unquantized`` (fp64 attention on the bf16 inputs, same rows) the error
+    against it is recorded too."""
+    st = attention_errors(got, want, rows)
+    total = st["n"] + st["n_excluded"]
+    uq = unquantized_errors(got, unquantized, rows) if unquantized is not None else None
+    RECORDS.append(dict(what=what, uq=uq, **st))
+    msg = (f"{what}: gated max {st['max']:.3e} mean {st['mean']:.3e} | plain max "
+           f"{st['plain_max']:.3e} mean {st['plain_mean']:.3e} | max|ref| {st['max_ref']:.3e} | "
+           f"{st['n']} outputs, {st['n_tie']} with a tie allowance, {st['n_excluded']} excluded "
+           f"(move decided at the threshold), {st['n_nonfinite_ok']} non-finite as the oracle, "
+           f"{st['n_nonfinite_bad']} non-finite mismatches")
+    if uq is not None:
+        msg += f" | vs unquantised fp64: max {uq[0]:.3e} mean {uq[1]:.3e}"
+    print(msg)
+    assert st["n_nonfinite_bad"] == 0, msg
+    assert st["max"] <= MAX_ABS_TOL and st["mean"] <= MEAN_ABS_TOL, msg
+    assert st["n_excluded"] <= MAX_EXCLUDED_FRACTION * max(total, 1), msg
+    return st["max"], st["mean"]

@@ -8,6 +8,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 from tests.conftest import ROOT
 
@@ -193,3 +194,35 @@ def test_plain_c_consumer(tmp_path):
                            "-L", lib_dir, "-lfp8attn", f"-Wl,-rpath,{lib_dir}", "-o", exe])
     r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout + r.stderr
+
+
+def test_noalloc_sources_checked_before_any_launch(monkeypatch):
+    """The allocation-free entry point runs the same host-side source checks
+    as Context.quantize_qkv: a total_tokens beyond the packed source's rows
+    and a padded layout whose sequences leave the source raise before the
+    library is called.  (CPU tensors stand in for device ones here; the
+    binding's device check is switched off and the library must not be
+    reached.)"""
+    import quantization_amax_reduce_b200 as qar
+
+    def no_launch():
+        raise AssertionError("the library was called")
+
+    monkeypatch.setattr(qar, "_require_cuda", lambda t, name: None)
+    monkeypatch.setattr(qar, "lib", no_launch)
+    q = torch.zeros(128, 2, 128, dtype=torch.bfloat16)
+    o = torch.zeros(129, 2, 128, dtype=torch.uint8)
+    ds = torch.zeros(3, dtype=torch.float32)
+    with pytest.raises(ValueError, match="source rows"):
+        qar.quantize_qkv_noalloc(q, q, q, [0, 100, 129], 100, o, o, o, ds, total_tokens=129)
+    padded = torch.zeros(2, 64, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="outside"):
+        # the second sequence has 70 rows but starts at row 64 of 128
+        qar.quantize_qkv_noalloc(padded, padded, padded, [0, 60, 130], 70, o, o, o, ds,
+                                 total_tokens=130, src_seq_start=[0, 64])
+    with pytest.raises(ValueError, match="total_tokens is required"):
+        qar.quantize_qkv_noalloc(padded, padded, padded, [0, 60, 120], 64, o, o, o, ds,
+                                 src_seq_start=[0, 64])
+    with pytest.raises(ValueError, match="needed"):
+        qar.quantize_qkv_noalloc(q, q, q, [0, 100, 128], 100, o, o, o,
+                                 torch.zeros(2, dtype=torch.float32))

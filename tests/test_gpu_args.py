@@ -46,3 +46,22 @@ def test_output_buffers_are_checked_before_launch():
         ctx.quantize_qkv(0, qar.DYNAMIC, q, k, v, cu_d, 100, total_tokens=129)
     # only the one good quantisation launched
     assert n1 == n0 + 1 and qar.launch_count() == n1
+
+
+def test_noalloc_checks_and_counts_its_launch():
+    """The allocation-free entry point refuses a total_tokens beyond the
+    source rows before launching, and a good call counts as one launch."""
+    q, k, v, cu = synthetic.small_qkv(4, [100, 28], H=2, device=DEV)
+    cu_d = torch.as_tensor(cu, device=DEV)
+    outs = [torch.zeros(129, 2, 128, dtype=torch.uint8, device=DEV) for _ in range(3)]
+    ds = torch.zeros(3, dtype=torch.float32, device=DEV)
+    n0 = qar.launch_count()
+    with pytest.raises(ValueError, match="source rows"):
+        qar.quantize_qkv_noalloc(q, k, v, cu_d, 100, *outs, ds, total_tokens=129)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        qar.quantize_qkv_noalloc(q, k, v, cu_d, 100, *outs, torch.zeros(3, dtype=torch.float32))
+    assert qar.launch_count() == n0
+    qar.quantize_qkv_noalloc(q, k, v, cu_d, 100, *outs, ds)
+    torch.cuda.synchronize()
+    assert qar.quantize_qkv_noalloc_error() == 0
+    assert qar.launch_count() == n0 + 1

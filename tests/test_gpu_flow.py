@@ -32,9 +32,21 @@ def test_c4_dit_dynamic_full_size():
     for g, w, n in zip((q8, k8, v8), codes, "qkv"):
         assert_codes_equal(g, w, n)
     assert_scales_equal(ctx, 0, ol)
+    ds = [float(x) for x in ol.ds]
+    # every head on a few rows ...
     rows = sample_rows(cu, 24, seed=4)
-    want = oracle.attention_fp8(*codes, cu, [float(x) for x in ol.ds], rows=rows, return_ambiguity=True)
-    assert_attention_close(out, want, rows=rows, what="c4")
+    want = oracle.attention_fp8(*codes, cu, ds, rows=rows, return_ambiguity=True)
+    assert_attention_close(out, want, rows=rows, what="c4 all heads")
+    # ... and 1024 rows of the first and the last head, with the error
+    # against unquantised fp64 attention on the bf16 inputs
+    heads = [0, 39]
+    rows = sample_rows(cu, 1024, seed=40)
+    sub = [np.ascontiguousarray(c[:, heads]) for c in codes]
+    want = oracle.attention_fp8(*sub, cu, ds, rows=rows, return_ambiguity=True)
+    ref = oracle.attention_bf16(*(np.ascontiguousarray(bits(x)[:, heads]) for x in (q, k, v)), cu,
+                                rows=rows)
+    assert_attention_close(out[:, heads], want, rows=rows, what="c4 1024 rows x 2 heads",
+                           unquantized=ref)
     assert ctx.get_error() == 0
 
 
@@ -91,12 +103,16 @@ def test_c5_calibrate_then_serve():
         cu_d = torch.as_tensor(cu, device=DEV)
         max_len = int(np.diff(cu).max())
         q, k, v, _ = synthetic.qkv(5, l, serve, device=DEV)
-        rows = sample_rows(cu, 16, seed=l)
+        # 1024 rows per sequence of two heads on the first FP8 layer served,
+        # 64 rows of every head on the others
+        many = l == min(check_layers)
+        rows = sample_rows(cu, 1024 if many else 64, seed=l)
+        heads = [0, w.H - 1] if many else list(range(w.H))
         mode = ctx.select_mode(l, mask)
         if mode == qar.SKIP:
             out = qar.varlen_fwd_bf16(q, k, v, cu_d, max_len)
             want = oracle.attention_bf16(bits(q), bits(k), bits(v), cu, rows=rows)
-            assert_attention_close(out, want, rows=rows, what=f"serve bf16 layer {l}")
+            assert_attention_close(out, want, rows=rows, what=f"c5 serve bf16 layer {l}")
             continue
         assert mode == qar.STATIC
         q8, k8, v8 = ctx.quantize_qkv(l, qar.STATIC, q, k, v, cu_d, max_len)
@@ -105,5 +121,11 @@ def test_c5_calibrate_then_serve():
             assert_codes_equal(g, ww, f"serve layer {l} {n}")
         assert_scales_equal(ctx, l, ols[l])
         out = qar.varlen_fwd(q8, k8, v8, cu_d, max_len, ctx.descale_ptr(l))
-        want = oracle.attention_fp8(*codes, cu, [float(x) for x in ols[l].ds], rows=rows, return_ambiguity=True)
-        assert_attention_close(out, want, rows=rows, what=f"serve fp8 layer {l}")
+        sub = [np.ascontiguousarray(c[:, heads]) for c in codes]
+        want = oracle.attention_fp8(*sub, cu, [float(x) for x in ols[l].ds], rows=rows,
+                                    return_ambiguity=True)
+        ref = oracle.attention_bf16(*(np.ascontiguousarray(bits(x)[:, heads]) for x in (q, k, v)),
+                                    cu, rows=rows)
+        assert_attention_close(out[:, heads], want, rows=rows,
+                               what=f"c5 serve fp8 layer {l} ({len(heads)} heads)",
+                               unquantized=ref)

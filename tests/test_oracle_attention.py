@@ -264,3 +264,117 @@ def test_ambiguity_reported_only_at_rounding_ties():
     o, amb = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True,
                                   return_ambiguity=True)
     assert (amb == 0.0).all()
+
+
+# --------------------------------------------------------------------------
+# The tie model: which codes an implementation may decide either way
+# --------------------------------------------------------------------------
+
+def _two_key_case_with_cancelling_channels(s1_code, big):
+    """_two_key_case, plus (when `big`) two more channels whose products
+    +448 and -448 cancel: the score is unchanged but sum |q_d k_d| (the
+    scale of the tensor cores' accumulation error) is ~900x larger."""
+    q8, k8, v8, cu = _two_key_case(s1_code)
+    if big:
+        q8[:, 0, 1] = 0x38
+        q8[:, 0, 2] = 0x38
+        k8[1, 0, 1] = 0x7E            # +448
+        k8[1, 0, 2] = 0xFE            # -448
+    return q8, k8, v8, cu
+
+
+def test_exp2_tie_window_grows_with_the_accumulation_scale():
+    # y1 = 32 exp(s1) = 29 (1 + 3e-5): 3e-5 above the tie between the E4M3
+    # values 28 and 30.  With the score's products all small the
+    # implementation's error is ~3e-6 relative and the code is decided; with
+    # two cancelling 448 x 1 products it may be off by ~3e-4, so either code
+    # is a correct result and an allowance is reported.
+    ds_k = math.log(29.0 * (1.0 + 3e-5) / 32.0)
+    for big, want_amb in ((False, False), (True, True)):
+        q8, k8, v8, cu = _two_key_case_with_cancelling_channels(0x38, big)
+        o, amb = oracle.attention_fp8(q8, k8, v8, cu, (1.0, ds_k, 1.0), scale=1.0,
+                                      return_ambiguity=True)
+        assert (amb[0, 0, 1] > 0) == want_amb, (big, amb[0, 0, 1])
+        assert abs(o[0, 0, 1] - (30.0 / 32.0) / (1.0 + 29.0 * (1 + 3e-5) / 32.0)) < 1e-12
+
+
+def test_linear_log_tie_window_grows_with_the_accumulation_scale():
+    # 8 t1 + 56 = 94.502: 0.002 code units above the half-integer between
+    # codes 94 and 95.  Small products: decided; cancelling 448 x 1 products:
+    # within the implementation's error, so an allowance is reported.
+    t1 = (94.502 - 56.0) / 8.0
+    ds_k = (t1 - 5.0) / math.log2(math.e)          # s1 = ds_k, r = 0
+    for big, want_amb in ((False, False), (True, True)):
+        q8, k8, v8, cu = _two_key_case_with_cancelling_channels(0x38, big)
+        o, amb = oracle.attention_fp8(q8, k8, v8, cu, (1.0, ds_k, 1.0), scale=1.0,
+                                      return_ambiguity=True, rule=oracle.P_LINEAR_LOG)
+        assert (amb[0, 0, 1] > 0) == want_amb, (big, amb[0, 0, 1])
+
+
+# --------------------------------------------------------------------------
+# The linear-log P rule: code = RNE(8 t + 56) clamped to [0, 128]
+# --------------------------------------------------------------------------
+
+def test_linear_log_code_interpolates_between_powers_of_two():
+    # t1 = 4.5 exactly (s1 = -ln(2)/2): 8 t + 56 = 92 = 0x5C, exponent field
+    # 11, mantissa 4: (1 + 4/8) 2^4 = 24, so p~1 = 24/32 = 0.75 (linear between
+    # 2^4 and 2^5) where the exp2 rule gives e4m3(22.63) = 22 -> 0.6875.
+    # Key 0 (score 0, the block max): 8 * 5 + 56 = 96 = 0x60 = 32 -> 1.
+    # l is the sum of the quantised values, 1 + 0.75.
+    q8, k8, v8, cu = _two_key_case(0x38)
+    ds_k = -0.5 * math.log(2.0)
+    o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, ds_k, 1.0), scale=1.0,
+                             rule=oracle.P_LINEAR_LOG)
+    assert abs(o[0, 0, 1] - 0.75 / 1.75) < 1e-15
+    e = oracle.attention_fp8(q8, k8, v8, cu, (1.0, ds_k, 1.0), scale=1.0)
+    assert abs(e[0, 0, 1] - 0.6875 / (1.0 + math.sqrt(0.5))) < 1e-15
+
+
+def test_linear_log_code_rounds_the_fraction_to_eighths():
+    # s1 = -0.125: t1 = 5 - 0.18034 = 4.81966, 8 t + 56 = 94.557 -> 95 = 0x5F:
+    # exponent 11, mantissa 7: (1 + 7/8) 16 = 30 -> p~1 = 30/32.
+    q8, k8, v8, cu = _two_key_case(0xA0)      # k1 = -0.125 e_0
+    o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0,
+                             rule=oracle.P_LINEAR_LOG)
+    assert abs(o[0, 0, 1] - (30.0 / 32.0) / (1.0 + 30.0 / 32.0)) < 1e-15
+
+
+def test_linear_log_subnormal_codes_and_the_clamp():
+    # s1 = -8: t1 = 5 - 11.5416 = -6.5416, 8 t + 56 = 3.667 -> code 4, an
+    # E4M3 subnormal: 4 * 2^-9 = 2^-7, so p~1 = 2^-7 / 32 = 2^-12.
+    q8, k8, v8, cu = _two_key_case(0xD0)      # k1 = -8 e_0
+    o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0,
+                             rule=oracle.P_LINEAR_LOG)
+    assert abs(o[0, 0, 1] - 2.0 ** -12 / (1.0 + 2.0 ** -12)) < 1e-18
+    # s1 = -20: 8 t + 56 < 0 -> code 0, the key drops out entirely
+    q8, k8, v8, cu = _two_key_case(0xDA)      # k1 = -20 e_0
+    o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0,
+                             rule=oracle.P_LINEAR_LOG)
+    assert o[0, 0, 1] == 0.0
+
+
+def test_linear_log_nan_score_gets_code_zero():
+    # a NaN key code makes that key's score NaN: its P code is 0, so the
+    # output is the other key's value exactly (v0 = e_2 here)
+    q8, k8, v8, cu = _two_key_case(0x7F)      # k1 = NaN
+    v8[0, 0, 2] = 0x38
+    o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0,
+                             rule=oracle.P_LINEAR_LOG)
+    assert o[0, 0, 2] == 1.0 and o[0, 0, 1] == 0.0
+
+
+def test_linear_log_rows_average_exactly():
+    # l is the sum of the quantised P, so with v = 1 every output is 1 (up
+    # to fp64 rounding), with the reference moving or not
+    H, D = 2, 128
+    lens = [300, 7]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(cu[-1])
+    g = torch.Generator().manual_seed(17)
+    ramp = torch.linspace(0.2, 3.0, T).view(T, 1, 1)
+    q8 = (torch.randn(T, H, D, generator=g) * 4).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    k8 = (torch.randn(T, H, D, generator=g) * 4 * ramp).to(torch.float8_e4m3fn).view(
+        torch.uint8).numpy()
+    ones = np.full((T, H, D), 0x38, np.uint8)
+    o = oracle.attention_fp8(q8, k8, ones, cu, (0.25, 0.25, 1.0), rule=oracle.P_LINEAR_LOG)
+    np.testing.assert_allclose(o, 1.0, rtol=0, atol=1e-13)
