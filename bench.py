@@ -11,10 +11,17 @@ attention kernel's microseconds and the fused quantise kernel's GB/s.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-N > 1 runs under torchrun, one rank per GPU, each rank its own independent
-copy of the workload (weak scaling, no collective on the data path); the
-reported time is the max over ranks.  ``--impl reference`` times the CPU
-oracle on the host cores on bounded samples of the same workload.
+With N > 1 and no torchrun environment the script starts its own N ranks
+(torch.distributed.run, one rank per GPU, NCCL).  Every rank times its own
+independent copy of the step (weak scaling, no collective on the data path;
+the reported time is the max over ranks), and then measures the one layer
+of the DiT-shaped workload (S=32760, 40 heads) split across the ranks the
+two ways the multi-GPU path supports: head-sharded dynamic quantisation (a
+3-float all-reduce MAX of the amax) with attention on the local heads, and a
+sequence-parallel (Ulysses) step with its two all-to-alls.  ``--dry-run``
+replaces the GPU work by a CPU stand-in on gloo ranks (launcher and
+aggregation checks).  ``--impl reference`` times the CPU oracle on the host
+cores on bounded samples of the same workload.
 """
 from __future__ import annotations
 
@@ -23,6 +30,7 @@ import hashlib
 import json
 import math
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -43,7 +51,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 FP8_PER_BF16 = 2.0                                    # nominal dense ratio (4.5 / 2.25 PF)
 ATTN_SOURCES = ["quantization_amax_reduce_b200/csrc/attention.cu",
                 "quantization_amax_reduce_b200/csrc/sm100_ptx.cuh"]
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_fp8_s8192_h16.md")
+QUANT_SOURCES = ["quantization_amax_reduce_b200/csrc/quant.cu",
+                 "quantization_amax_reduce_b200/csrc/sm100_ptx.cuh",
+                 "quantization_amax_reduce_b200/csrc/state.cuh"]
+PROFILES = os.path.join(ROOT, "profiles")
+P_RULES = {"linear_log": 0, "exp2": 1}
 
 
 def parse_args(argv=None):
@@ -57,6 +69,12 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-dynamic-quant", action="store_true",
                    help="skip the separate dynamic-quantisation measurement")
+    p.add_argument("--no-per-config", action="store_true",
+                   help="skip the per-workload attention timings and error figures")
+    p.add_argument("--p-rule", choices=sorted(P_RULES), default="linear_log",
+                   help="P quantisation rule of the FP8 attention (fp8attn_p_rule)")
+    p.add_argument("--dry-run", action="store_true",
+                   help="CPU stand-in for the GPU work on gloo ranks (launcher checks)")
     return p.parse_args(argv)
 
 
@@ -101,23 +119,20 @@ def source_digest(paths) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
-    """DRAM bytes per attention launch from the committed ncu summary, or None
-    when the kernel sources changed since it was captured."""
-    if not os.path.exists(PROFILE_SUMMARY):
-        return None
-    vals = {}
-    with open(PROFILE_SUMMARY) as f:
-        for line in f:
-            if ":" in line and line.strip().startswith("- "):
-                k, v = line.strip()[2:].split(":", 1)
-                vals[k.strip()] = v.strip().strip("`")
-    try:
-        if vals.get("source_digest") != source_digest(ATTN_SOURCES):
-            return None
-        return float(vals["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
+def profiled_traffic(name: str, sources):
+    """DRAM bytes per launch of a kernel from its committed ncu summary
+    (profiles/<name>.json), or None when the kernel's sources changed since
+    the capture.  Returns (bytes, label)."""
+    path = os.path.join(PROFILES, name + ".json")
+    if not os.path.exists(path):
+        return None, None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("source_digest") != source_digest(sources):
+        return None, None
+    label = (f"ncu capture {name}.json ({d.get('capture', 'one launch')}, SM clock "
+             f"{d.get('sm_clock_ghz', '?')} GHz)")
+    return float(d["dram_bytes_per_launch"]), label
 
 
 class ClockSampler:
@@ -338,6 +353,274 @@ def measure_dynamic_quant(dev, stream, reps: int = 20):
             "kernel": "quant_dynamic_kernel"}
 
 
+def _time_launches(fn, dev, stream, reps: int, flush=None):
+    """Median device time (s) of `fn` over `reps` launches, each after an L2
+    flush when `flush` is given (events on the launching stream)."""
+    import torch
+    ts = []
+    for _ in range(reps):
+        if flush is not None:
+            flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        ts.append(a.elapsed_time(b) / 1e3)
+    return statistics.median(ts)
+
+
+def _unquantized_reference(q, k, v, cu, rows, heads):
+    """fp64 softmax attention on the bf16 inputs (CPU, plain torch) for the
+    given global query rows and heads: the figure the error against
+    unquantised attention is taken from."""
+    import numpy as np
+    import torch
+    out = torch.empty((len(rows), len(heads), D), dtype=torch.float64)
+    cu = np.asarray(cu)
+    for n, r in enumerate(rows):
+        b = int(np.searchsorted(cu, r, side="right") - 1)
+        s0, s1 = int(cu[b]), int(cu[b + 1])
+        for m, h in enumerate(heads):
+            qq = q[r, h].double()
+            kk = k[s0:s1, h].double()
+            vv = v[s0:s1, h].double()
+            p = torch.softmax(kk @ qq / math.sqrt(D), dim=0)
+            out[n, m] = p @ vv
+    return out
+
+
+def _err_vs_unquantized(out, q, k, v, cu, rows, heads):
+    import torch
+    ref = _unquantized_reference(q.cpu(), k.cpu(), v.cpu(), cu, rows, heads)
+    got = out.cpu()[rows][:, heads].double()
+    d = (got - ref).abs()
+    return {"max": float(d.max()), "mean": float(d.mean()), "rows": len(rows),
+            "heads": list(heads)}
+
+
+def _sample_rows(cu, per_seq, seed):
+    import numpy as np
+    rng = np.random.Generator(np.random.PCG64(seed))
+    rows = []
+    for b in range(len(cu) - 1):
+        s0, s1 = int(cu[b]), int(cu[b + 1])
+        n = s1 - s0
+        pick = {0, n - 1, (n - 1) // 128 * 128}
+        pick.update(rng.choice(n, size=min(per_seq, n), replace=False).tolist())
+        rows.extend(s0 + x for x in sorted(pick))
+    return sorted(set(rows))
+
+
+def measure_per_config(dev, stream, p_rule, fp8_peak, flush):
+    """Attention time, throughput and roofline fraction of the other
+    workloads (outside the timed step), and the error of the FP8 path
+    against unquantised fp64 attention on sampled rows."""
+    import torch
+
+    import synthetic
+    import quantization_amax_reduce_b200 as qar
+
+    res = {}
+
+    def attn_entry(name, q8, k8, v8, cu, cu_d, max_len, ds_ptr, flops, q, k, v, rows, heads,
+                   reps):
+        T, Hn = q8.shape[0], q8.shape[1]
+        out = torch.empty((T, Hn, D), dtype=torch.bfloat16, device=dev)
+
+        def run():
+            qar.varlen_fwd(q8, k8, v8, cu_d, max_len, ds_ptr, out=out, stream=stream,
+                           p_rule=p_rule)
+        run()
+        sec = _time_launches(run, dev, stream, reps, flush)
+        tf = flops / sec / 1e12
+        res[name] = {"attn_us": sec * 1e6, "attn_tflops": tf, "frac": tf / fp8_peak,
+                     "flops": flops, "err_vs_unquantized": _err_vs_unquantized(
+                         out, q, k, v, cu, rows, heads)}
+
+    # config 2: ViT-shaped varlen batch after its 16 dynamic passes
+    w = synthetic.WORKLOADS[2]
+    cu = w.cu_seqlens(0)
+    cu_d = torch.as_tensor(cu, device=dev)
+    max_len = int(max(w.seq_lens(0)))
+    ctx = qar.Context(1, device=dev)
+    for p in range(w.passes):
+        q, k, v, _ = synthetic.qkv(2, 0, p, device=dev)
+        q8, k8, v8 = ctx.quantize_qkv(0, qar.DYNAMIC, q, k, v, cu_d, max_len, stream=stream)
+    attn_entry("vit_varlen3_h16_after_16_passes", q8, k8, v8, cu, cu_d, max_len,
+               ctx.descale_ptr(0), w.flops(0), q, k, v, _sample_rows(cu, 6, 2), [0, 15], 10)
+    res["vit_varlen3_h16_after_16_passes"]["seq_lens"] = w.seq_lens(0)
+    del q, k, v, q8, k8, v8
+
+    # config 4: DiT-shaped single sequence, dynamic pass
+    w = synthetic.WORKLOADS[4]
+    q, k, v, cu = synthetic.qkv(4, device=dev)
+    cu_d = torch.as_tensor(cu, device=dev)
+    ctx = qar.Context(1, device=dev)
+    q8, k8, v8 = ctx.quantize_qkv(0, qar.DYNAMIC, q, k, v, cu_d, 32760, stream=stream)
+    attn_entry("dit_s32760_h40_dynamic", q8, k8, v8, cu, cu_d, 32760, ctx.descale_ptr(0),
+               w.flops(0), q, k, v, _sample_rows(cu, 8, 4), [0, 39], 5)
+    del q, k, v, q8, k8, v8
+
+    # config 5: one served layer (layer 3 of 24, dynamic pass on its inputs)
+    w = synthetic.WORKLOADS[5]
+    cu = w.cu_seqlens(3)
+    cu_d = torch.as_tensor(cu, device=dev)
+    max_len = int(max(w.seq_lens(3)))
+    q, k, v, _ = synthetic.qkv(5, 3, 0, device=dev)
+    ctx = qar.Context(1, device=dev)
+    q8, k8, v8 = ctx.quantize_qkv(0, qar.DYNAMIC, q, k, v, cu_d, max_len, stream=stream)
+    attn_entry("calibrate_serve_layer3_varlen4_h16", q8, k8, v8, cu, cu_d, max_len,
+               ctx.descale_ptr(0), w.flops(3), q, k, v, _sample_rows(cu, 4, 5), [0, 15], 5)
+    res["calibrate_serve_layer3_varlen4_h16"]["seq_lens"] = w.seq_lens(3)
+    if ctx.get_error() != 0:
+        raise RuntimeError("device error in the per-workload runs")
+    return res
+
+
+def measure_sharded(dev, stream, rank, world, dist, p_rule, reps: int = 5):
+    """One layer of the DiT-shaped workload (S=32760, 40 heads) split across
+    the ranks.  (a) Head-sharded: this rank's 40/N heads, dynamic amax of the
+    local heads -> all-reduce MAX of 3 floats -> ring push -> cast with the
+    ring scales -> FP8 attention of the local heads.  (b) Sequence-parallel
+    (Ulysses): this rank's S/N tokens of all heads, quantised before the
+    all-to-all.  Times are device times, max over ranks."""
+    import torch
+
+    import synthetic
+    import quantization_amax_reduce_b200 as qar
+
+    S4, H4 = 32760, 40
+    if H4 % world or S4 % world:
+        return None
+    q, k, v, cu = synthetic.qkv(4, device=dev)
+    Hn, Sn = H4 // world, S4 // world
+    hs = slice(rank * Hn, (rank + 1) * Hn)
+    ql, kl, vl = q[:, hs], k[:, hs], v[:, hs]
+    cu_d = torch.as_tensor(cu, device=dev)
+    ctx = qar.Context(1, device=dev)
+    comm = qar.TorchComm()
+    codes = tuple(torch.empty((S4, Hn, D), dtype=torch.uint8, device=dev) for _ in range(3))
+    out = torch.empty((S4, Hn, D), dtype=torch.bfloat16, device=dev)
+    amax = torch.empty(3, dtype=torch.float32, device=dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+
+    def head_step():
+        ev[0].record(stream)
+        ctx.amax_qkv(ql, kl, vl, cu_d, S4, out=amax, stream=stream)
+        ev[1].record(stream)
+        comm.all_reduce_max(amax)
+        ev[2].record(stream)
+        ctx.amax_ring_update(0, amax, stream=stream)
+        ctx.quantize_qkv(0, qar.RING, ql, kl, vl, cu_d, S4, out=codes, stream=stream)
+        qar.varlen_fwd(*codes, cu_d, S4, ctx.descale_ptr(0), out=out, stream=stream,
+                       p_rule=p_rule)
+        ev[3].record(stream)
+
+    for _ in range(2):
+        head_step()
+    torch.cuda.synchronize(dev)
+    step_s, xchg_s = [], []
+    for _ in range(reps):
+        dist.barrier()
+        head_step()
+        torch.cuda.synchronize(dev)
+        step_s.append(ev[0].elapsed_time(ev[3]) / 1e3)
+        xchg_s.append(ev[1].elapsed_time(ev[2]) / 1e3)
+    head_max = max_over_ranks(statistics.median(step_s), dist, dev)
+    xchg_max = max_over_ranks(statistics.median(xchg_s), dist, dev)
+
+    # sequence-parallel step over this rank's tokens
+    ctx_u = qar.Context(1, device=dev)
+    tok = slice(rank * Sn, (rank + 1) * Sn)
+    qu, ku, vu = (x[tok].contiguous() for x in (q, k, v))
+    del q, k, v
+    ua, ub = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def uly_step():
+        return qar.ulysses_attention(ctx_u, 0, qar.DYNAMIC, qu, ku, vu, comm=comm,
+                                     p_rule=p_rule)
+    for _ in range(2):
+        uly_step()
+    torch.cuda.synchronize(dev)
+    us = []
+    for _ in range(reps):
+        dist.barrier()
+        ua.record(torch.cuda.current_stream(dev))
+        uly_step()
+        ub.record(torch.cuda.current_stream(dev))
+        torch.cuda.synchronize(dev)
+        us.append(ua.elapsed_time(ub) / 1e3)
+    uly_max = max_over_ranks(statistics.median(us), dist, dev)
+    if ctx.get_error() != 0 or ctx_u.get_error() != 0:
+        raise RuntimeError("device error in the sharded runs")
+    flops = 4.0 * S4 * S4 * D * H4
+    return {
+        "workload": "dit_s32760_h40 one layer, dynamic, split over the ranks",
+        "head_sharded": {"heads_per_rank": Hn, "step_us": head_max * 1e6,
+                         "tflops": flops / head_max / 1e12,
+                         "allreduce_us": xchg_max * 1e6,
+                         "exchange_share": xchg_max / head_max},
+        "ulysses": {"tokens_per_rank": Sn, "step_us": uly_max * 1e6,
+                    "tflops": flops / uly_max / 1e12},
+    }
+
+
+def run_dry(args):
+    """CPU stand-in for the GPU work (gloo): checks the launcher, the
+    max-over-ranks timing and the aggregation without a GPU."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if world > 1:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    a = torch.randn(128, 128)
+    for _ in range(args.warmup):
+        a @ a
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        a = torch.tanh(a @ a)
+    secs = time.perf_counter() - t0 + 0.01 * rank       # ranks differ on purpose
+    slowest = max_over_ranks(secs, dist if world > 1 else None, torch.device("cpu"))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": aggregate_throughput(args.steps, world, slowest),
+            "unit": "steps/s (dry run)", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": slowest / max(args.steps, 1) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "dry_run": True,
+            "config": {"workload": "cpu stand-in", "parallelism": f"{world} gloo ranks"}}))
+    return 0
+
+
+def _free_port() -> int:
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def spawn_ranks(args, argv) -> int:
+    """Start N ranks of this script under torch.distributed.run (one per
+    GPU; rendezvous on 127.0.0.1).  Rank 0 prints the JSON line."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr=127.0.0.1",
+           f"--master-port={_free_port()}", os.path.abspath(__file__)] + list(argv)
+    env = dict(os.environ, OMP_NUM_THREADS=os.environ.get("OMP_NUM_THREADS", "4"))
+    try:
+        return subprocess.run(cmd, env=env, timeout=3600).returncode
+    except subprocess.TimeoutExpired:
+        return 124
+
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -368,8 +651,10 @@ def run_ours(args):
     def quant():
         ctx.quantize_qkv(0, qar.STATIC, q, k, v, cu_d, S, out=(q8, k8, v8), stream=stream)
 
+    p_rule = P_RULES[args.p_rule]
+
     def attn():
-        qar.varlen_fwd(q8, k8, v8, cu_d, S, ds_ptr, out=out, stream=stream)
+        qar.varlen_fwd(q8, k8, v8, cu_d, S, ds_ptr, out=out, stream=stream, p_rule=p_rule)
 
     # L2 flush between timed steps: read a 256 MB buffer (> 126 MB of L2), so
     # the next step starts with a cold cache and no dirty lines to write back
@@ -451,7 +736,7 @@ def run_ours(args):
                 s_comp.wait_event(ev_out[i - 2])       # output buffer b downloaded
             ctx.quantize_qkv(0, qar.STATIC, dq[b], dk[b], dv[b], cu_d, S, out=d8[b],
                              stream=s_comp)
-            qar.varlen_fwd(*d8[b], cu_d, S, ds_ptr, out=dout[b], stream=s_comp)
+            qar.varlen_fwd(*d8[b], cu_d, S, ds_ptr, out=dout[b], stream=s_comp, p_rule=p_rule)
             ev_comp[i].record(s_comp)
             s_out.wait_event(ev_comp[i])
             with torch.cuda.stream(s_out):
@@ -470,11 +755,29 @@ def run_ours(args):
         raise RuntimeError("device error during the end-to-end steps")
 
     dyn = None if args.no_dynamic_quant else measure_dynamic_quant(dev, stream)
+    peaks, src = load_peaks()
+    fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
+
+    # this workload's error against unquantised fp64 attention, and the
+    # attention time under the other P rule (outside the timed step)
+    err_uq = _err_vs_unquantized(out, q, k, v, cu, _sample_rows(cu, 24, 3), list(range(H)))
+    other = "exp2" if args.p_rule == "linear_log" else "linear_log"
+
+    def attn_other():
+        qar.varlen_fwd(q8, k8, v8, cu_d, S, ds_ptr, out=out, stream=stream,
+                       p_rule=P_RULES[other])
+    attn_other()
+    other_s = _time_launches(attn_other, dev, stream, 20, flush_l2)
+    per_config = None
+    if world == 1 and not args.no_per_config:
+        per_config = measure_per_config(dev, stream, p_rule, fp8_peak, flush_l2)
+    sharded = measure_sharded(dev, stream, rank, world, dist, p_rule) if world > 1 else None
 
     result = None
     if rank == 0:
-        peaks, src = load_peaks()
-        fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
+        attn_traffic, attn_traffic_src = profiled_traffic("attn_fp8_s8192_h16", ATTN_SOURCES)
+        quant_traffic, quant_traffic_src = profiled_traffic("quant_static_s8192_h16",
+                                                            QUANT_SOURCES)
         attn_s = statistics.mean(attn_ms) / 1e3
         quant_s = statistics.mean(quant_ms) / 1e3
         attn_tflops = FLOPS_PER_STEP / attn_s / 1e12
@@ -488,16 +791,22 @@ def run_ours(args):
             "data": "synthetic",
             "config": {"workload": WORKLOAD, "S": S, "heads": H, "head_dim": D, "batch": 1,
                        "scales": "static q=224 k=198 v=210", "l2": "flushed between steps",
-                       "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"},
+                       "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU",
+                       "p_rule": args.p_rule},
+            "p_rule": args.p_rule,
             "attn_us": attn_s * 1e6, "attn_tflops": attn_tflops,
+            "attn_other_rule": {"p_rule": other, "attn_us": other_s * 1e6,
+                                "attn_tflops": FLOPS_PER_STEP / other_s / 1e12},
+            "err_vs_unquantized": err_uq,
             "quant_us": quant_s * 1e6, "quant_gbs": quant_gbs,
             "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": fp8_peak,
                          "unit": "TFLOP/s", "frac": attn_tflops / fp8_peak,
-                         "traffic": profiled_traffic(),
+                         "traffic": attn_traffic, "traffic_source": attn_traffic_src,
                          "kernel": "attn_fwd_fp8_kernel",
                          "peak_source": f"{src} bf16 burst x{FP8_PER_BF16:g} (fp8/bf16 nominal)"},
             "quant_roofline": {"bound": "hbm", "achieved": quant_gbs, "peak": peaks["hbm_gbs"],
                                "unit": "GB/s", "frac": quant_gbs / peaks["hbm_gbs"],
+                               "traffic": quant_traffic, "traffic_source": quant_traffic_src,
                                "kernel": "quant_static_kernel", "peak_source": src},
             "kernel_share": {"attn_fwd_fp8_kernel": share_attn,
                              "quant_static_kernel": 1.0 - share_attn},
@@ -512,7 +821,18 @@ def run_ours(args):
             dyn["frac"] = dyn["gbs_algorithmic"] / peaks["hbm_gbs"]
             dyn["peak"] = peaks["hbm_gbs"]
             dyn["peak_source"] = src
+            dyn_bytes, dyn_src = profiled_traffic("quant_dynamic_s32760_h40", QUANT_SOURCES)
+            if dyn_bytes is not None:
+                # the same kernel against the DRAM bytes ncu counted
+                dyn["dram_bytes"] = dyn_bytes
+                dyn["gbs_dram"] = dyn_bytes / (dyn["us"] * 1e-6) / 1e9
+                dyn["frac_dram"] = dyn["gbs_dram"] / peaks["hbm_gbs"]
+                dyn["traffic_source"] = dyn_src
             result["quant_dynamic"] = dyn
+        if per_config is not None:
+            result["per_config"] = per_config
+        if sharded is not None:
+            result["sharded"] = sharded
         if clocks is not None:
             result["clocks"] = clocks
     if world > 1:
@@ -526,7 +846,12 @@ def run_ours(args):
 
 
 def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
     args = parse_args(argv)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return spawn_ranks(args, argv)
+    if args.dry_run:
+        return run_dry(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

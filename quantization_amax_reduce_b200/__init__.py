@@ -689,7 +689,7 @@ def _single_seq_cu(S: int, device) -> torch.Tensor:
 
 def ulysses_attention(ctx: "Context", layer: int, mode: int, q: torch.Tensor, k: torch.Tensor,
                       v: torch.Tensor, comm=None, softmax_scale: float = 0.0,
-                      stream=None) -> torch.Tensor:
+                      stream=None, p_rule: int = P_EXP2) -> torch.Tensor:
     """Sequence-parallel (Ulysses) attention over one sequence whose tokens are
     split evenly across the ranks of ``comm`` (a :class:`TorchComm` by
     default): rank r holds tokens [r S_loc, (r+1) S_loc) of Q, K, V as bf16
@@ -755,7 +755,7 @@ def ulysses_attention(ctx: "Context", layer: int, mode: int, q: torch.Tensor, k:
             o = varlen_fwd_bf16(recv[0], recv[1], recv[2], cu_all, S, softmax_scale)
         else:
             o = varlen_fwd(recv[0], recv[1], recv[2], cu_all, S, ctx.descale_ptr(layer),
-                           softmax_scale)
+                           softmax_scale, p_rule=p_rule)
         if n == 1:
             return o.view(S_loc, H, D)
         back = torch.empty_like(o)

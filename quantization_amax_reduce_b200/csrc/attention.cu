@@ -484,7 +484,8 @@ struct Fp8Barriers {
   uint64_t q_full;
   uint64_t k_full[Fp8Cfg::kStages];
   uint64_t v_full[Fp8Cfg::kStages];
-  uint64_t kv_empty[Fp8Cfg::kStages];
+  uint64_t k_empty[Fp8Cfg::kStages];   // the S products that read the K stage are done
+  uint64_t v_empty[Fp8Cfg::kStages];   // the PV products that read the V stage are done
   uint64_t s_full[2];       // S_i of the current block computed
   uint64_t s_free[2];       // S_i loaded by the softmax (TMEM columns free)
   uint64_t p_full[2][2];    // [tile][P buffer] P_i written
@@ -533,7 +534,8 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&bars.k_full[s], 1);
       mbar_init(&bars.v_full[s], 1);
-      mbar_init(&bars.kv_empty[s], 1);
+      mbar_init(&bars.k_empty[s], 1);
+      mbar_init(&bars.v_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.s_full[i], 1);
@@ -568,30 +570,56 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
       for (int i = 0; i < 2; ++i)
         tma_load_3d(sq + i * C::kTile, &tm_q, &bars.q_full, 0, h, seq0 + q0 + 128 * i);
     }
-    int issued = 0;
-    for (int j = 0; j < nkv; ++j) {
-      const int st = j % C::kStages;
-      if (j >= C::kStages) {
-        if (!mbar_wait(&bars.kv_empty[st], ((j / C::kStages) - 1) & 1, abort_flag)) {
-          if (leader) note_error(p, bars, kErrTimeout);
-          break;
+    // K and V stages are released separately: a K stage as soon as the two
+    // S products that read it are done, a V stage after its PV products.  K
+    // therefore streams up to kStages blocks ahead of the S products while V
+    // follows the (later) PV products; the producer polls both without
+    // blocking, keeping V no further ahead than K.
+    int jk = 0, jv = 0;
+    uint64_t t_last = global_timer_ns();
+    uint32_t polls = 0;
+    bool ok = true;
+    while (jv < nkv) {
+      bool progressed = false;
+      if (jk < nkv) {
+        const int st = jk % C::kStages;
+        if (jk < C::kStages || mbar_test(&bars.k_empty[st], ((jk / C::kStages) - 1) & 1)) {
+          if (leader) {
+            mbar_expect_tx(&bars.k_full[st], C::kTile);
+            tma_load_3d(sk + st * C::kTile, &tm_k, &bars.k_full[st], 0, h, seq0 + 128 * jk);
+          }
+          ++jk;
+          progressed = true;
         }
       }
-      if (leader) {
-        const int tok = seq0 + 128 * j;
-        mbar_expect_tx(&bars.k_full[st], C::kTile);
-        tma_load_3d(sk + st * C::kTile, &tm_k, &bars.k_full[st], 0, h, tok);
-        mbar_expect_tx(&bars.v_full[st], C::kTile);
-        tma_load_3d(sv + st * C::kTile, &tm_v, &bars.v_full[st], 0, h, tok);
+      if (jv < jk) {
+        const int st = jv % C::kStages;
+        if (jv < C::kStages || mbar_test(&bars.v_empty[st], ((jv / C::kStages) - 1) & 1)) {
+          if (leader) {
+            mbar_expect_tx(&bars.v_full[st], C::kTile);
+            tma_load_3d(sv + st * C::kTile, &tm_v, &bars.v_full[st], 0, h, seq0 + 128 * jv);
+          }
+          ++jv;
+          progressed = true;
+        }
       }
       __syncwarp();
-      issued = j + 1;
+      if (progressed) {
+        polls = 0;
+        t_last = 0;
+      } else if ((++polls & 63u) == 0) {
+        // bounded like every other wait: give up after kWaitLimitNs without progress
+        const uint64_t now = global_timer_ns();
+        if (t_last == 0) t_last = now;
+        if (*abort_flag || now - t_last > kWaitLimitNs) { ok = false; break; }
+      }
     }
-    for (int j = (issued > C::kStages ? issued - C::kStages : 0); j < issued; ++j) {
-      const int st = j % C::kStages;
-      mbar_wait(&bars.k_full[st], (j / C::kStages) & 1, nullptr);
-      mbar_wait(&bars.v_full[st], (j / C::kStages) & 1, nullptr);
-    }
+    if (!ok && leader) note_error(p, bars, kErrTimeout);
+    // make sure no copy is still landing when the CTA leaves
+    for (int j = (jk > C::kStages ? jk - C::kStages : 0); j < jk; ++j)
+      mbar_wait(&bars.k_full[j % C::kStages], (j / C::kStages) & 1, nullptr);
+    for (int j = (jv > C::kStages ? jv - C::kStages : 0); j < jv; ++j)
+      mbar_wait(&bars.v_full[j % C::kStages], (j / C::kStages) & 1, nullptr);
     mbar_wait(&bars.q_full, 0, nullptr);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -642,6 +670,8 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
       tc_fence_after();
       issue_s(0, 0);
       issue_s(1, 0);
+      if (elect_one()) mma_commit(&bars.k_empty[0]);
+      __syncwarp();
     }
     for (int j = 0; j < nkv && ok; ++j) {
       const int st = j % C::kStages;
@@ -656,6 +686,9 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
           issue_s(i, j + 1);
         }
         if (!ok) break;
+        // K stage st1 is free once both S products of block j + 1 are done
+        if (elect_one()) mma_commit(&bars.k_empty[st1]);
+        __syncwarp();
       }
       ok = mbar_wait(&bars.v_full[st], (j / C::kStages) & 1, abort_flag);
       if (ok && j + 1 == nkv && (len & 127)) zero_tail_rows(sv + st * C::kTile, len & 127, lane);
@@ -666,7 +699,7 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         issue_pv(i, j);
       }
       if (!ok) break;
-      if (elect_one()) mma_commit(&bars.kv_empty[st]);
+      if (elect_one()) mma_commit(&bars.v_empty[st]);
       __syncwarp();
     }
     if (!ok && leader) note_error(p, bars, kErrTimeout);

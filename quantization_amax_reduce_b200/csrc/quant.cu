@@ -257,6 +257,12 @@ __global__ void __launch_bounds__(kThreads) quant_dynamic_kernel(QuantArgs a) {
 // become the layer's current scales), or the ring's current scales as left by
 // the last ring update (a shard of a head-sharded pass, whose amax was
 // reduced across ranks and pushed with fp8attn_amax_ring_update).
+// Q, K and V are swept together: each step of a thread reads the same two
+// 16-byte vectors (16 channels of one token and head) of all three tensors
+// and writes three 16-byte code vectors, so the whole launch is one grid
+// stride loop with six loads in flight per step and no per-tensor tail.
+constexpr int kUnrollStatic = 2;
+
 template <bool kContig>
 __global__ void __launch_bounds__(kThreads) quant_static_kernel(QuantArgs a) {
   if (!seqlens_ok(a)) {
@@ -264,9 +270,37 @@ __global__ void __launch_bounds__(kThreads) quant_static_kernel(QuantArgs a) {
     return;
   }
   const int64_t T = __ldg(a.cu + a.B);
-  const int64_t nvec = T * a.H * 16;
-  const float* qs = a.cast_with_ring ? a.ls->qs : a.ls->static_qs;
-  for (int t = 0; t < 3; ++t) cast_sweep<kContig>(a, t, nvec, qs[t], false);
+  const int64_t npair = T * a.H * 8;   // pairs of 16-byte vectors (16 rows of a channel block)
+  const float* qsp = a.cast_with_ring ? a.ls->qs : a.ls->static_qs;
+  const float qs[3] = {qsp[0], qsp[1], qsp[2]};
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t p0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; p0 < npair;
+       p0 += stride * kUnrollStatic) {
+    uint4 x[kUnrollStatic][3][2];
+#pragma unroll
+    for (int u = 0; u < kUnrollStatic; ++u) {
+      const int64_t p = p0 + u * stride;
+      // vectors 2p and 2p + 1 lie in the same 128-channel row, 8 elements apart
+      const int64_t off = p < npair ? src_offset<kContig>(a, 2 * p) : 0;
+#pragma unroll
+      for (int t = 0; t < 3; ++t) {
+        x[u][t][0] = p < npair ? ld_vec(a.src[t] + off) : make_uint4(0, 0, 0, 0);
+        x[u][t][1] = p < npair ? ld_vec(a.src[t] + off + 8) : make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnrollStatic; ++u) {
+      const int64_t p = p0 + u * stride;
+      if (p < npair) {
+#pragma unroll
+        for (int t = 0; t < 3; ++t) {
+          const uint2 lo = cast8(x[u][t][0], qs[t]);
+          const uint2 hi = cast8(x[u][t][1], qs[t]);
+          reinterpret_cast<uint4*>(a.dst[t])[p] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+        }
+      }
+    }
+  }
   if (!a.cast_with_ring && blockIdx.x == 0 && threadIdx.x < 3) {
     a.ls->qs[threadIdx.x] = a.ls->static_qs[threadIdx.x];
     a.ls->ds[threadIdx.x] = a.ls->static_ds[threadIdx.x];

@@ -30,8 +30,9 @@ def _finite_codes(rng, shape):
 def _tiles(seed):
     """Six kinds of 128 x 128 tile pairs, 4 of each."""
     rng = np.random.default_rng(seed)
-    enc = lambda x: torch.from_numpy(x.astype(np.float32)).to(torch.float8_e4m3fn).view(
-        torch.uint8).numpy()
+    # values are clipped to the E4M3 range first (torch maps larger ones to NaN)
+    enc = lambda x: torch.from_numpy(np.clip(x, -448.0, 448.0).astype(np.float32)).to(
+        torch.float8_e4m3fn).view(torch.uint8).numpy()
     qs, ks = [], []
     for kind in range(6):
         for _ in range(4):

@@ -60,3 +60,27 @@ def test_single_rank_identity():
     import bench
     assert bench.max_over_ranks(3.5, None) == 3.5
     assert bench.aggregate_throughput(10.0, 1, 2.0) == 5.0
+
+
+def test_bench_starts_its_own_ranks_and_aggregates():
+    """`python bench.py --gpus 2` without a torchrun environment starts two
+    ranks itself; --dry-run replaces the GPU work by a CPU stand-in on gloo,
+    so the launcher, the max-over-ranks time and the whole-job aggregate are
+    checked here without a GPU."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2",
+                        "--dry-run", "--steps", "5", "--warmup", "1"],
+                       capture_output=True, text=True, timeout=300, env=env, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout            # rank 0 alone prints
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and d["dry_run"] and d["steps"] == 5
+    # whole-job throughput: both ranks' steps over the slowest rank's time
+    slowest = d["ms_per_step"] * d["steps"] / 1e3
+    assert abs(d["value"] - 2 * 5 / slowest) < 1e-6 * d["value"]
