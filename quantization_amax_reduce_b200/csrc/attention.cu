@@ -480,6 +480,12 @@ struct Fp8Cfg {
   static constexpr int kSmemBytes = (2 + 2 * kStages + 4) * kTile + 1024 + 1024;
 };
 
+// FP8 kernel warps: 0-7 softmax, 8 TMA producer, 9 and 10 MMA issuers for
+// query tiles 0 and 1 (each on its own SM sub-partition, so the two issue
+// streams and their barrier waits overlap instead of queueing behind each
+// other; each tile's MMAs still complete in issue order).
+constexpr int kThreadsFp8 = 352;
+
 struct Fp8Barriers {
   uint64_t q_full;
   uint64_t k_full[Fp8Cfg::kStages];
@@ -490,13 +496,14 @@ struct Fp8Barriers {
   uint64_t s_free[2];       // S_i loaded by the softmax (TMEM columns free)
   uint64_t p_full[2][2];    // [tile][P buffer] P_i written
   uint64_t pv_done[2][2];   // [tile][P buffer] PV_i that read that buffer done
-  uint64_t drain;
+  uint64_t v_tail;          // the last, partial V tile's rows past the sequence are zeroed
+  uint64_t drain[2];
   uint32_t tmem_base;
   int abort_flag;
 };
 
 template <int kRule>
-__global__ void __launch_bounds__(kThreadsAttn, 1)
+__global__ void __launch_bounds__(kThreadsFp8, 1)
 attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, AttnParams p) {
@@ -534,8 +541,8 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&bars.k_full[s], 1);
       mbar_init(&bars.v_full[s], 1);
-      mbar_init(&bars.k_empty[s], 1);
-      mbar_init(&bars.v_empty[s], 1);
+      mbar_init(&bars.k_empty[s], 2);   // one commit per MMA warp
+      mbar_init(&bars.v_empty[s], 2);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.s_full[i], 1);
@@ -545,7 +552,9 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_init(&bars.pv_done[i][q], 1);
       }
     }
-    mbar_init(&bars.drain, 1);
+    mbar_init(&bars.v_tail, 1);
+    mbar_init(&bars.drain[0], 1);
+    mbar_init(&bars.drain[1], 1);
     bars.abort_flag = 0;
     fence_mbar_init();
   }
@@ -583,7 +592,7 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
       bool progressed = false;
       if (jk < nkv) {
         const int st = jk % C::kStages;
-        if (jk < C::kStages || mbar_test(&bars.k_empty[st], ((jk / C::kStages) - 1) & 1)) {
+        if (jk < C::kStages || mbar_test_now(&bars.k_empty[st], ((jk / C::kStages) - 1) & 1)) {
           if (leader) {
             mbar_expect_tx(&bars.k_full[st], C::kTile);
             tma_load_3d(sk + st * C::kTile, &tm_k, &bars.k_full[st], 0, h, seq0 + 128 * jk);
@@ -594,7 +603,7 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       if (jv < jk) {
         const int st = jv % C::kStages;
-        if (jv < C::kStages || mbar_test(&bars.v_empty[st], ((jv / C::kStages) - 1) & 1)) {
+        if (jv < C::kStages || mbar_test_now(&bars.v_empty[st], ((jv / C::kStages) - 1) & 1)) {
           if (leader) {
             mbar_expect_tx(&bars.v_full[st], C::kTile);
             tma_load_3d(sv + st * C::kTile, &tm_v, &bars.v_full[st], 0, h, seq0 + 128 * jv);
@@ -621,19 +630,20 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int j = (jv > C::kStages ? jv - C::kStages : 0); j < jv; ++j)
       mbar_wait(&bars.v_full[j % C::kStages], (j / C::kStages) & 1, nullptr);
     mbar_wait(&bars.q_full, 0, nullptr);
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
+    // ------------------------------------------------------------ MMA issuers
+    const int i = warp - kMmaWarp;   // query tile of this warp
     const bool leader = lane == 0;
     const uint32_t id_qk = make_idesc(0, 0, 128, 0);
     const uint32_t id_pv = make_idesc(0, 0, 128, 1);
-    const uint64_t dq0 = make_sdesc_sw128(smem_u32(sq), 16, 1024);
+    const uint64_t dq = make_sdesc_sw128(smem_u32(sq), 16, 1024) + static_cast<uint64_t>(i * (C::kTile >> 4));
     const uint64_t dk0 = make_sdesc_sw128(smem_u32(sk), 16, 1024);
     const uint64_t dv0 = make_sdesc_sw128(smem_u32(sv), 16384, 1024);
     const uint64_t dp0 = make_sdesc_sw128(smem_u32(sp), 16, 1024);
     constexpr uint32_t kStep = C::kTile >> 4;
-    auto issue_s = [&](int i, int j) {
+    const uint32_t tS = tmem + 128 * i, tO = tmem + 256 + 128 * i;
+    auto issue_s = [&](int j) {
       uint64_t ad[4], bd[4];
-      const uint64_t dq = dq0 + static_cast<uint64_t>(i * kStep);
       const uint64_t dk = dk0 + static_cast<uint64_t>((j % C::kStages) * kStep);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
@@ -642,12 +652,14 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tmem + 128 * i, ad[kk], bd[kk], id_qk, kk > 0);
+        for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tS, ad[kk], bd[kk], id_qk, kk > 0);
         mma_commit(&bars.s_full[i]);
+        // the K stage is free once both tiles' S products of block j are done
+        mma_commit(&bars.k_empty[j % C::kStages]);
       }
       __syncwarp();
     };
-    auto issue_pv = [&](int i, int j) {
+    auto issue_pv = [&](int j) {
       uint64_t ad[4], bd[4];
       const uint64_t dp = dp0 + static_cast<uint64_t>((2 * i + (j & 1)) * kStep);
       const uint64_t dv = dv0 + static_cast<uint64_t>((j % C::kStages) * kStep);
@@ -659,53 +671,48 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint32_t acc0 = j > 0 ? 1u : 0u;
       if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_f8_ss(tmem + 256 + 128 * i, ad[kk], bd[kk], id_pv, kk > 0 ? 1u : acc0);
+        for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tO, ad[kk], bd[kk], id_pv, kk > 0 ? 1u : acc0);
         mma_commit(&bars.pv_done[i][j & 1]);
+        mma_commit(&bars.v_empty[j % C::kStages]);
       }
       __syncwarp();
     };
     bool ok = mbar_wait(&bars.q_full, 0, abort_flag) && mbar_wait(&bars.k_full[0], 0, abort_flag);
     if (ok) {
       tc_fence_after();
-      issue_s(0, 0);
-      issue_s(1, 0);
-      if (elect_one()) mma_commit(&bars.k_empty[0]);
-      __syncwarp();
+      issue_s(0);
     }
     for (int j = 0; j < nkv && ok; ++j) {
       const int st = j % C::kStages;
       if (j + 1 < nkv) {
         const int st1 = (j + 1) % C::kStages;
-        ok = mbar_wait(&bars.k_full[st1], ((j + 1) / C::kStages) & 1, abort_flag);
-        for (int i = 0; i < 2 && ok; ++i) {
-          // S_i's TMEM columns are free once the softmax has loaded block j
-          ok = mbar_wait(&bars.s_free[i], j & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          issue_s(i, j + 1);
-        }
-        if (!ok) break;
-        // K stage st1 is free once both S products of block j + 1 are done
-        if (elect_one()) mma_commit(&bars.k_empty[st1]);
-        __syncwarp();
-      }
-      ok = mbar_wait(&bars.v_full[st], (j / C::kStages) & 1, abort_flag);
-      if (ok && j + 1 == nkv && (len & 127)) zero_tail_rows(sv + st * C::kTile, len & 127, lane);
-      for (int i = 0; i < 2 && ok; ++i) {
-        ok = mbar_wait(&bars.p_full[i][j & 1], (j >> 1) & 1, abort_flag);
+        // S_i's TMEM columns are free once the softmax has loaded block j
+        ok = mbar_wait(&bars.k_full[st1], ((j + 1) / C::kStages) & 1, abort_flag) &&
+             mbar_wait(&bars.s_free[i], j & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        issue_pv(i, j);
+        issue_s(j + 1);
       }
+      ok = mbar_wait(&bars.v_full[st], (j / C::kStages) & 1, abort_flag);
+      if (ok && j + 1 == nkv && (len & 127)) {
+        // tile 0's warp zeroes the rows past the sequence; tile 1's waits for it
+        if (i == 0) {
+          zero_tail_rows(sv + st * C::kTile, len & 127, lane);
+          if (leader) mbar_arrive(&bars.v_tail);
+        } else {
+          ok = mbar_wait(&bars.v_tail, 0, abort_flag);
+        }
+      }
+      ok = ok && mbar_wait(&bars.p_full[i][j & 1], (j >> 1) & 1, abort_flag);
       if (!ok) break;
-      if (elect_one()) mma_commit(&bars.v_empty[st]);
-      __syncwarp();
+      tc_fence_after();
+      issue_pv(j);
     }
     if (!ok && leader) note_error(p, bars, kErrTimeout);
-    if (elect_one()) mma_commit(&bars.drain);
+    // drain: every MMA this warp issued has completed before TMEM is freed
+    if (elect_one()) mma_commit(&bars.drain[i]);
     __syncwarp();
-    mbar_wait(&bars.drain, 0, nullptr);
+    mbar_wait(&bars.drain[i], 0, nullptr);
   } else {
     // ------------------------------------------------------------ softmax
     const int wg = warp >> 2;
@@ -1039,7 +1046,8 @@ cudaError_t launch_attention_t(const AttnLaunch& a, int64_t T, cudaStream_t stre
   const int64_t grid = static_cast<int64_t>(p.n_qblk) * a.heads * a.batch;
   if (grid <= 0) return cudaSuccess;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
-  kernel<<<static_cast<unsigned>(grid), kThreadsAttn, smem_bytes, stream>>>(mq, mk, mv, p);
+  kernel<<<static_cast<unsigned>(grid), kFp8 ? kThreadsFp8 : kThreadsAttn, smem_bytes, stream>>>(
+      mq, mk, mv, p);
   return cudaGetLastError();
 }
 

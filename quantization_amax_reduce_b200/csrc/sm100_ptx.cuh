@@ -77,6 +77,35 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of a phase (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_now(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait_limit spinning on test_wait (no suspension at all): for a warp
+// whose waits are usually already satisfied and whose latency matters.
+__device__ __forceinline__ bool mbar_spin_limit(uint64_t* bar, uint32_t parity,
+                                                const volatile int* abort_flag,
+                                                uint64_t limit_ns) {
+  if (mbar_test_now(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_test_now(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (abort_flag && *abort_flag) return false;
+      if (global_timer_ns() - t0 > limit_ns) return false;
+    }
+  }
+}
+
 // Wait until the phase with the given parity has completed.  Returns false
 // if the wait ran past `limit_ns` or `abort_flag` (shared memory, may be
 // null) became non-zero.  Spins on try_wait (no suspend hint: a suspended
