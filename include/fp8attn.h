@@ -236,8 +236,10 @@ typedef enum {
 } fp8attn_p_rule;
 
 /* fp8attn_varlen_fwd with an explicit P rule (fp8attn_varlen_fwd uses
- * FP8ATTN_P_EXP2).  Errors as fp8attn_varlen_fwd, and INVALID for an unknown
- * rule. */
+ * FP8ATTN_P_LINEAR_LOG, which evaluates no exponential per score and is the
+ * faster of the two on B200, where the exponential unit is otherwise the
+ * bottleneck; FP8ATTN_P_EXP2 rounds the exact exponential).  Errors as
+ * fp8attn_varlen_fwd, and INVALID for an unknown rule. */
 fp8attn_status fp8attn_varlen_fwd_rule(const void* q8, const void* k8, const void* v8,
                                        const int32_t* d_cu_seqlens, int batch, int max_seqlen,
                                        int64_t total_tokens, int num_heads, int head_dim,

@@ -229,7 +229,7 @@ P_LINEAR_LOG, P_EXP2 = "linear_log", "exp2"
 
 def attention_fp8(q8, k8, v8, cu, ds_qkv: Sequence[float], scale: Optional[float] = None,
                   pquant: bool = True, l_of_quantized: bool = False, rows=None,
-                  nthreads: int = 0, return_ambiguity: bool = False, rule: str = P_EXP2):
+                  nthreads: int = 0, return_ambiguity: bool = False, rule: str = P_LINEAR_LOG):
     """fp64 attention on E4M3 codes [T, H, D]; returns [len(rows) or T, H, D].
 
     With ``pquant`` the PV product uses P quantised per block of 128 keys (in

@@ -407,11 +407,12 @@ def _attn_common(q, k, v, cu_seqlens, out, dtype):
 def varlen_fwd(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, cu_seqlens,
                max_seqlen: int, descale, softmax_scale: float = 0.0,
                out: Optional[torch.Tensor] = None, error: Optional[torch.Tensor] = None,
-               stream=None, p_rule: int = P_EXP2) -> torch.Tensor:
+               stream=None, p_rule: int = P_LINEAR_LOG) -> torch.Tensor:
     """FP8 attention on packed E4M3 [T, H, 128] codes.  ``descale`` is a device
     pointer (int, e.g. ``Context.descale_ptr(layer)``) or a 3-element fp32 CUDA
     tensor {ds_q, ds_k, ds_v}.  ``p_rule`` picks how P is quantised for the PV
-    product (P_EXP2 or P_LINEAR_LOG, see fp8attn_p_rule in fp8attn.h).
+    product (P_LINEAR_LOG, the default, or P_EXP2; see fp8attn_p_rule in
+    fp8attn.h).
     Returns bf16 [T, H, 128]."""
     T, H, cu, out = _attn_common(q8, k8, v8, cu_seqlens, out, torch.uint8)
     if isinstance(descale, torch.Tensor):
@@ -689,7 +690,7 @@ def _single_seq_cu(S: int, device) -> torch.Tensor:
 
 def ulysses_attention(ctx: "Context", layer: int, mode: int, q: torch.Tensor, k: torch.Tensor,
                       v: torch.Tensor, comm=None, softmax_scale: float = 0.0,
-                      stream=None, p_rule: int = P_EXP2) -> torch.Tensor:
+                      stream=None, p_rule: int = P_LINEAR_LOG) -> torch.Tensor:
     """Sequence-parallel (Ulysses) attention over one sequence whose tokens are
     split evenly across the ranks of ``comm`` (a :class:`TorchComm` by
     default): rank r holds tokens [r S_loc, (r+1) S_loc) of Q, K, V as bf16

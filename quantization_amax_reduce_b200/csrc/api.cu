@@ -377,7 +377,7 @@ fp8attn_status fp8attn_varlen_fwd(const void* q8, const void* k8, const void* v8
                                   int32_t* d_error, void* stream) {
   return run_attention(q8, k8, v8, d_cu_seqlens, batch, max_seqlen, total_tokens, num_heads,
                        head_dim, d_descale_qkv, softmax_scale, out, d_error, stream, 0,
-                       FP8ATTN_P_EXP2);
+                       FP8ATTN_P_LINEAR_LOG);
 }
 
 fp8attn_status fp8attn_varlen_fwd_rule(const void* q8, const void* k8, const void* v8,

@@ -21,6 +21,10 @@ pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
 
+# both P rules of the FP8 kernel, each against the oracle's statement of it
+RULES = [pytest.param(qar.P_LINEAR_LOG, oracle.P_LINEAR_LOG, id="linear_log"),
+         pytest.param(qar.P_EXP2, oracle.P_EXP2, id="exp2")]
+
 
 def _codes(T, H, seed, scale=1.0):
     g = torch.Generator().manual_seed(seed)
@@ -38,8 +42,9 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("rule,orule", RULES)
 @pytest.mark.parametrize("lens,H", CASES)
-def test_fp8_attention_small_shapes(lens, H):
+def test_fp8_attention_small_shapes(lens, H, rule, orule):
     cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
     T = int(cu[-1])
     q8, k8, v8 = (_codes(T, H, s, 6.0) for s in (1, 2, 3))
@@ -47,9 +52,10 @@ def test_fp8_attention_small_shapes(lens, H):
     # absolute tolerance measures the kernel rather than bf16 output rounding
     ds = torch.tensor([0.05, 0.04, 1.0 / 60.0], dtype=torch.float32)
     out = qar.varlen_fwd(q8.to(DEV), k8.to(DEV), v8.to(DEV), torch.as_tensor(cu, device=DEV),
-                         max(lens), ds.to(DEV))
-    want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds.tolist(), return_ambiguity=True)
-    assert_attention_close(out, want, what=f"fp8 {lens} H={H}")
+                         max(lens), ds.to(DEV), p_rule=rule)
+    want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds.tolist(),
+                                return_ambiguity=True, rule=orule)
+    assert_attention_close(out, want, what=f"fp8 {lens} H={H} {orule}")
 
 
 @pytest.mark.parametrize("lens,H", CASES[:8])
@@ -63,7 +69,8 @@ def test_bf16_attention_small_shapes(lens, H):
     assert_attention_close(out, want, what=f"bf16 {lens} H={H}")
 
 
-def test_sharp_softmax_rescales():
+@pytest.mark.parametrize("rule,orule", RULES)
+def test_sharp_softmax_rescales(rule, orule):
     """Large score range so the reference max moves across key tiles (O
     rescaling in TMEM) and many p fall in E4M3's subnormal range."""
     lens = [900]
@@ -77,36 +84,42 @@ def test_sharp_softmax_rescales():
     v8 = (torch.randn(900, H, 128, generator=g) * 4).to(torch.float8_e4m3fn).view(torch.uint8)
     ds = [0.25, 0.25, 0.025]
     out = qar.varlen_fwd(q8.to(DEV), k8.to(DEV), v8.to(DEV), torch.as_tensor(cu, device=DEV),
-                         900, torch.tensor(ds, device=DEV))
-    want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds, return_ambiguity=True)
-    assert_attention_close(out, want, what="sharp")
+                         900, torch.tensor(ds, device=DEV), p_rule=rule)
+    want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds, return_ambiguity=True,
+                                rule=orule)
+    assert_attention_close(out, want, what=f"sharp {orule}")
 
 
-def test_explicit_softmax_scale():
+@pytest.mark.parametrize("rule,orule", RULES)
+def test_explicit_softmax_scale(rule, orule):
     cu = np.array([0, 300], dtype=np.int32)
     q8, k8, v8 = (_codes(300, 2, s, 3.0) for s in (4, 5, 6))
     ds = [0.1, 0.1, 0.05]
     out = qar.varlen_fwd(q8.to(DEV), k8.to(DEV), v8.to(DEV), torch.as_tensor(cu, device=DEV),
-                         300, torch.tensor(ds, device=DEV), softmax_scale=0.3)
-    want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds, scale=0.3, return_ambiguity=True)
-    assert_attention_close(out, want, what="scale 0.3")
+                         300, torch.tensor(ds, device=DEV), softmax_scale=0.3, p_rule=rule)
+    want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds, scale=0.3,
+                                return_ambiguity=True, rule=orule)
+    assert_attention_close(out, want, what=f"scale 0.3 {orule}")
 
 
-def test_c1_end_to_end_through_the_boundary():
+@pytest.mark.parametrize("rule,orule", RULES)
+def test_c1_end_to_end_through_the_boundary(rule, orule):
     q, k, v, cu = synthetic.qkv(1)
     ctx = qar.Context(1)
     cu_d = torch.as_tensor(cu, device=DEV)
     q8, k8, v8 = ctx.quantize_qkv(0, qar.DYNAMIC, q.to(DEV), k.to(DEV), v.to(DEV), cu_d, 256)
-    out = qar.varlen_fwd(q8, k8, v8, cu_d, 256, ctx.descale_ptr(0))
+    out = qar.varlen_fwd(q8, k8, v8, cu_d, 256, ctx.descale_ptr(0), p_rule=rule)
     ol = OracleLayer()
     codes = ol.dynamic_pass([bits(q), bits(k), bits(v)], cu, 2)
-    want = oracle.attention_fp8(*codes, cu, [float(x) for x in ol.ds], return_ambiguity=True)
+    want = oracle.attention_fp8(*codes, cu, [float(x) for x in ol.ds], return_ambiguity=True,
+                                rule=orule)
     # the error against unquantised fp64 attention on the bf16 inputs is reported
     ref = oracle.attention_bf16(bits(q), bits(k), bits(v), cu)
-    assert_attention_close(out, want, what="c1", unquantized=ref)
+    assert_attention_close(out, want, what=f"c1 {orule}", unquantized=ref)
 
 
-def test_c3_full_size_sampled_rows():
+@pytest.mark.parametrize("rule,orule", RULES)
+def test_c3_full_size_sampled_rows(rule, orule):
     """The benchmarked configuration: S=8192, 16 heads, static 224/198/210.
     The oracle quantises the bf16 inputs itself (codes and scales must equal
     the kernel's bit for bit) and attends on its own codes."""
@@ -115,7 +128,7 @@ def test_c3_full_size_sampled_rows():
     ctx.set_static_scales(0, 224.0, 198.0, 210.0)
     cu_d = torch.as_tensor(cu, device=DEV)
     q8, k8, v8 = ctx.quantize_qkv(0, qar.STATIC, q, k, v, cu_d, 8192)
-    out = qar.varlen_fwd(q8, k8, v8, cu_d, 8192, ctx.descale_ptr(0))
+    out = qar.varlen_fwd(q8, k8, v8, cu_d, 8192, ctx.descale_ptr(0), p_rule=rule)
     ol = OracleLayer()
     ol.set_static([224.0, 198.0, 210.0])
     hq, hk, hv = bits(q), bits(k), bits(v)
@@ -125,12 +138,13 @@ def test_c3_full_size_sampled_rows():
     assert_scales_equal(ctx, 0, ol)
     rows = sample_rows(cu, 192, seed=3)
     want = oracle.attention_fp8(*codes, cu, [float(x) for x in ol.ds], rows=rows,
-                                return_ambiguity=True)
+                                return_ambiguity=True, rule=orule)
     ref = oracle.attention_bf16(hq, hk, hv, cu, rows=rows)
-    assert_attention_close(out, want, rows=rows, what="c3", unquantized=ref)
+    assert_attention_close(out, want, rows=rows, what=f"c3 {orule}", unquantized=ref)
 
 
-def test_c2_varlen_after_sixteen_passes_sampled_rows():
+@pytest.mark.parametrize("rule,orule", RULES)
+def test_c2_varlen_after_sixteen_passes_sampled_rows(rule, orule):
     """Config 2 after its 16 dynamic passes: the oracle follows the ring
     through every pass, quantises the last pass itself and attends on its
     own codes."""
@@ -154,12 +168,12 @@ def test_c2_varlen_after_sixteen_passes_sampled_rows():
         assert_codes_equal(g, ww, n)
     assert_scales_equal(ctx, 0, ol)
     assert_ring_equal(ctx, 0, ol)
-    out = qar.varlen_fwd(q8, k8, v8, cu_d, max_len, ctx.descale_ptr(0))
+    out = qar.varlen_fwd(q8, k8, v8, cu_d, max_len, ctx.descale_ptr(0), p_rule=rule)
     rows = sample_rows(cu, 128, seed=2)
     want = oracle.attention_fp8(*codes, cu, [float(x) for x in ol.ds], rows=rows,
-                                return_ambiguity=True)
+                                return_ambiguity=True, rule=orule)
     ref = oracle.attention_bf16(hq, hk, hv, cu, rows=rows)
-    assert_attention_close(out, want, rows=rows, what="c2", unquantized=ref)
+    assert_attention_close(out, want, rows=rows, what=f"c2 {orule}", unquantized=ref)
 
 
 def _nan_boundary_case(kind):
@@ -190,7 +204,8 @@ def _nan_boundary_case(kind):
     return lens, H, cu, q, k, v
 
 
-def test_fp8_nan_in_the_next_sequence_does_not_leak():
+@pytest.mark.parametrize("rule,orule", RULES)
+def test_fp8_nan_in_the_next_sequence_does_not_leak(rule, orule):
     """A NaN code in sequence b+1 within the last, partial key tile of
     sequence b: sequence b must match the oracle (which attends only to its
     own keys), and the sequences holding NaN must be NaN exactly where the
@@ -198,13 +213,14 @@ def test_fp8_nan_in_the_next_sequence_does_not_leak():
     lens, H, cu, q8, k8, v8 = _nan_boundary_case("fp8")
     ds = [0.05, 0.04, 1.0 / 60.0]
     out = qar.varlen_fwd(q8.to(DEV), k8.to(DEV), v8.to(DEV), torch.as_tensor(cu, device=DEV),
-                         max(lens), torch.tensor(ds, device=DEV))
+                         max(lens), torch.tensor(ds, device=DEV), p_rule=rule)
     want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds,
-                                return_ambiguity=True)
+                                return_ambiguity=True, rule=orule)
     seq0 = np.arange(cu[0], cu[1])
     assert np.isfinite(out[:cu[1]].float().cpu().numpy()).all()
-    assert_attention_close(out, (want[0][seq0], want[1][seq0]), rows=seq0, what="fp8 NaN next")
-    assert_attention_close(out, want, what="fp8 NaN all")
+    assert_attention_close(out, (want[0][seq0], want[1][seq0]), rows=seq0,
+                           what=f"fp8 NaN next {orule}")
+    assert_attention_close(out, want, what=f"fp8 NaN all {orule}")
 
 
 def test_bf16_inf_and_nan_in_the_next_sequence_do_not_leak():
@@ -230,7 +246,8 @@ def test_bad_cu_seqlens_sets_error_word():
     assert qar.read_error_word(err) == 0
 
 
-def test_reference_max_stays_and_moves_by_design():
+@pytest.mark.parametrize("rule,orule", RULES)
+def test_reference_max_stays_and_moves_by_design(rule, orule):
     """Block maxima chosen so the reference max stays within the lag (block 1:
     +1.5 = +2.16 in log2 units), moves past it (block 2: +3.0 over the
     reference = +4.33), stays again (block 3), and sees a lower block (4);
@@ -248,8 +265,8 @@ def test_reference_max_stays_and_moves_by_design():
     q8, k8, v8 = (t.to(torch.float8_e4m3fn).view(torch.uint8) for t in (q, k, v))
     ds = [1.0, 1.0, 1.0]
     out = qar.varlen_fwd(q8.to(DEV), k8.to(DEV), v8.to(DEV), torch.as_tensor(cu, device=DEV), n,
-                         torch.tensor(ds, device=DEV), softmax_scale=1.0)
+                         torch.tensor(ds, device=DEV), softmax_scale=1.0, p_rule=rule)
     want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds, scale=1.0,
-                                return_ambiguity=True)
+                                return_ambiguity=True, rule=orule)
     assert np.isfinite(want[1]).all()                         # no decision at a tie
-    assert_attention_close(out, want, what="reference max stays and moves")
+    assert_attention_close(out, want, what=f"reference max stays and moves {orule}")

@@ -21,12 +21,14 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def test_c4_dit_dynamic_full_size():
+@pytest.mark.parametrize("rule,orule", [(qar.P_LINEAR_LOG, oracle.P_LINEAR_LOG),
+                                        (qar.P_EXP2, oracle.P_EXP2)], ids=["linear_log", "exp2"])
+def test_c4_dit_dynamic_full_size(rule, orule):
     q, k, v, cu = synthetic.qkv(4, device=DEV)
     ctx = qar.Context(1)
     cu_d = torch.as_tensor(cu, device=DEV)
     q8, k8, v8 = ctx.quantize_qkv(0, qar.DYNAMIC, q, k, v, cu_d, 32760)
-    out = qar.varlen_fwd(q8, k8, v8, cu_d, 32760, ctx.descale_ptr(0))
+    out = qar.varlen_fwd(q8, k8, v8, cu_d, 32760, ctx.descale_ptr(0), p_rule=rule)
     ol = OracleLayer()
     codes = ol.dynamic_pass([bits(q), bits(k), bits(v)], cu, 40)
     for g, w, n in zip((q8, k8, v8), codes, "qkv"):
@@ -35,17 +37,17 @@ def test_c4_dit_dynamic_full_size():
     ds = [float(x) for x in ol.ds]
     # every head on a few rows ...
     rows = sample_rows(cu, 24, seed=4)
-    want = oracle.attention_fp8(*codes, cu, ds, rows=rows, return_ambiguity=True)
-    assert_attention_close(out, want, rows=rows, what="c4 all heads")
+    want = oracle.attention_fp8(*codes, cu, ds, rows=rows, return_ambiguity=True, rule=orule)
+    assert_attention_close(out, want, rows=rows, what=f"c4 all heads {orule}")
     # ... and 1024 rows of the first and the last head, with the error
     # against unquantised fp64 attention on the bf16 inputs
     heads = [0, 39]
     rows = sample_rows(cu, 1024, seed=40)
     sub = [np.ascontiguousarray(c[:, heads]) for c in codes]
-    want = oracle.attention_fp8(*sub, cu, ds, rows=rows, return_ambiguity=True)
+    want = oracle.attention_fp8(*sub, cu, ds, rows=rows, return_ambiguity=True, rule=orule)
     ref = oracle.attention_bf16(*(np.ascontiguousarray(bits(x)[:, heads]) for x in (q, k, v)), cu,
                                 rows=rows)
-    assert_attention_close(out[:, heads], want, rows=rows, what="c4 1024 rows x 2 heads",
+    assert_attention_close(out[:, heads], want, rows=rows, what=f"c4 1024 rows x 2 heads {orule}",
                            unquantized=ref)
     assert ctx.get_error() == 0
 

@@ -48,7 +48,7 @@ def test_unquantized_p_matches_library_softmax(lens):
     q8, k8, v8 = (_codes((T, H, D), s, 2.0) for s in (1, 2, 3))
     ds = (0.031, 0.07, 1.7)
     scale = 1.0 / math.sqrt(D)
-    got = oracle.attention_fp8(q8, k8, v8, cu, ds, pquant=False)
+    got = oracle.attention_fp8(q8, k8, v8, cu, ds, pquant=False, rule=oracle.P_EXP2)
     want = _softmax_attention(_decode_torch(q8) * ds[0], _decode_torch(k8) * ds[1],
                               _decode_torch(v8) * ds[2], cu, scale)
     np.testing.assert_allclose(got, want, rtol=1e-11, atol=1e-13)
@@ -70,7 +70,7 @@ def test_zero_query_gives_mean_of_v_exactly_even_with_pquant():
     q8 = np.zeros((T, H, D), np.uint8)
     k8, v8 = _codes((T, H, D), 4), _codes((T, H, D), 5)
     ds_v = 0.75
-    got = oracle.attention_fp8(q8, k8, v8, cu, (0.5, 0.5, ds_v), pquant=True)
+    got = oracle.attention_fp8(q8, k8, v8, cu, (0.5, 0.5, ds_v), pquant=True, rule=oracle.P_EXP2)
     mean_v = _decode_torch(v8).mean(axis=0) * ds_v
     for t in range(T):
         np.testing.assert_allclose(got[t], mean_v, rtol=1e-14, atol=1e-15)
@@ -80,7 +80,7 @@ def test_single_key_returns_that_value():
     H, D = 3, 128
     cu = np.array([0, 1, 2], dtype=np.int32)        # two sequences of length 1
     q8, k8, v8 = (_codes((2, H, D), s, 3.0) for s in (6, 7, 8))
-    got = oracle.attention_fp8(q8, k8, v8, cu, (1.3, 0.2, 0.4), pquant=True)
+    got = oracle.attention_fp8(q8, k8, v8, cu, (1.3, 0.2, 0.4), pquant=True, rule=oracle.P_EXP2)
     np.testing.assert_array_equal(got, _decode_torch(v8) * 0.4)
 
 
@@ -102,15 +102,15 @@ def test_pquant_rule_normal_range():
     # [16, 32) where E4M3 spacing is 2, nearest 28 -> p~1 = 28/32 = 0.875.
     # l is the unquantised sum 1 + e^-0.125.
     q8, k8, v8, cu = _two_key_case(0xA0)      # 0xA0 = -0.125
-    o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True)
+    o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True, rule=oracle.P_EXP2)
     want = 0.875 / (1.0 + math.exp(-0.125))
     assert abs(o[0, 0, 1] - want) < 1e-15
     assert o[0, 0, 0] == 0.0
     # the unquantised and the "l = sum p~" variants differ visibly
-    o_none = oracle.attention_fp8(q8, k8, v8, cu, (1, 1, 1), scale=1.0, pquant=False)
+    o_none = oracle.attention_fp8(q8, k8, v8, cu, (1, 1, 1), scale=1.0, pquant=False, rule=oracle.P_EXP2)
     assert abs(o_none[0, 0, 1] - math.exp(-0.125) / (1 + math.exp(-0.125))) < 1e-15
     o_lq = oracle.attention_fp8(q8, k8, v8, cu, (1, 1, 1), scale=1.0, pquant=True,
-                                l_of_quantized=True)
+                                l_of_quantized=True, rule=oracle.P_EXP2)
     assert abs(o_lq[0, 0, 1] - 0.875 / 1.875) < 1e-15
 
 
@@ -119,7 +119,7 @@ def test_pquant_rule_subnormal_range():
     # the subnormal range with spacing 2^-9: 0.010735 / 2^-9 = 5.496 rounds
     # to 5, so p~1 = 5 * 2^-9 / 32 = 5 * 2^-14.
     q8, k8, v8, cu = _two_key_case(0xD0)      # 0xD0 = -8.0
-    o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True)
+    o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True, rule=oracle.P_EXP2)
     want = 5 * 2.0 ** -14 / (1.0 + math.exp(-8.0))
     assert abs(o[0, 0, 1] - want) < 1e-18
 
@@ -131,13 +131,13 @@ def test_rows_sum_to_one_and_columns_stay_in_range():
     T = int(cu[-1])
     q8, k8, v8 = (_codes((T, H, D), s, 4.0) for s in (10, 11, 12))
     ones = np.full((T, H, D), 0x38, np.uint8)
-    o = oracle.attention_fp8(q8, k8, ones, cu, (0.3, 0.3, 1.0), pquant=False)
+    o = oracle.attention_fp8(q8, k8, ones, cu, (0.3, 0.3, 1.0), pquant=False, rule=oracle.P_EXP2)
     np.testing.assert_allclose(o, 1.0, rtol=0, atol=1e-14)
-    oq = oracle.attention_fp8(q8, k8, ones, cu, (0.3, 0.3, 1.0), pquant=True)
+    oq = oracle.attention_fp8(q8, k8, ones, cu, (0.3, 0.3, 1.0), pquant=True, rule=oracle.P_EXP2)
     # |p~ - p| <= p / 16 for normal codes; a subnormal code is off by at most
     # half its 2^-9 step, 2^-10 / 32 = 2^-15 per key
     assert np.all(np.abs(oq - 1.0) <= 2.0 ** -4 + 64 * 2.0 ** -15)
-    o = oracle.attention_fp8(q8, k8, v8, cu, (0.3, 0.3, 1.0), pquant=False)
+    o = oracle.attention_fp8(q8, k8, v8, cu, (0.3, 0.3, 1.0), pquant=False, rule=oracle.P_EXP2)
     vv = _decode_torch(v8)
     for b in range(len(lens)):
         sl = slice(cu[b], cu[b + 1])
@@ -149,9 +149,9 @@ def test_row_subset_equals_full_rows():
     H, D = 2, 128
     cu = np.array([0, 20, 33], dtype=np.int32)
     q8, k8, v8 = (_codes((33, H, D), s, 2.0) for s in (13, 14, 15))
-    full = oracle.attention_fp8(q8, k8, v8, cu, (0.1, 0.2, 0.3))
+    full = oracle.attention_fp8(q8, k8, v8, cu, (0.1, 0.2, 0.3), rule=oracle.P_EXP2)
     rows = [0, 19, 20, 32, 5]
-    sub = oracle.attention_fp8(q8, k8, v8, cu, (0.1, 0.2, 0.3), rows=rows)
+    sub = oracle.attention_fp8(q8, k8, v8, cu, (0.1, 0.2, 0.3), rows=rows, rule=oracle.P_EXP2)
     np.testing.assert_array_equal(sub, full[rows])
 
 
@@ -177,7 +177,7 @@ def test_reference_max_stays_when_block_max_is_within_the_lag():
     # exact -> p~ = e^-1.  l = 128 e^-1 + 1 (unquantised).
     q8, k8, v8, cu = _block_step_case(0x38)          # s_128 = 1.0
     o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True,
-                             rows=[5])
+                             rows=[5], rule=oracle.P_EXP2)
     l = 128 * math.exp(-1.0) + 1.0
     assert abs(o[0, 0, 1] - 88.0 / 32.0 * math.exp(-1.0) / l) < 1e-15
     assert abs(o[0, 0, 2] - math.exp(-1.0) / l) < 1e-15
@@ -191,7 +191,7 @@ def test_reference_max_moves_past_the_lag():
     # (32 exactly) and carry e^-2.5.  l = 128 e^-2.5 + 1.
     q8, k8, v8, cu = _block_step_case(0x42)          # 0x42 = 2.5
     o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True,
-                             rows=[5])
+                             rows=[5], rule=oracle.P_EXP2)
     l = 128 * math.exp(-2.5) + 1.0
     assert abs(o[0, 0, 1] - 1.0 / l) < 1e-15
     assert abs(o[0, 0, 2] - math.exp(-2.5) / l) < 1e-15
@@ -204,10 +204,10 @@ def test_reference_move_at_the_threshold_makes_the_row_unverifiable():
     # a correct result of the rule, so the row's allowance is infinite
     q8, k8, v8, cu = _block_step_case(0x38)
     o, amb = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 3.0 * math.log(2.0), 1.0), scale=1.0,
-                                  pquant=True, rows=[5], return_ambiguity=True)
+                                  pquant=True, rows=[5], return_ambiguity=True, rule=oracle.P_EXP2)
     assert np.isinf(amb).all()
     o, amb = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 2.5, 1.0), scale=1.0,
-                                  pquant=True, rows=[5], return_ambiguity=True)
+                                  pquant=True, rows=[5], return_ambiguity=True, rule=oracle.P_EXP2)
     assert np.isfinite(amb).all()
 
 
@@ -226,7 +226,7 @@ def test_pquant_block_is_128_keys():
     v8[0, 0, 2] = 0x38                # v_0 = e_2
     cu = np.array([0, n], dtype=np.int32)
     o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True,
-                             rows=[0])
+                             rows=[0], rule=oracle.P_EXP2)
     l = 64 * math.exp(-1.0) + 1.0
     assert abs(o[0, 0, 2] - 0.375 / l) < 1e-15
 
@@ -243,7 +243,7 @@ def test_pquant_block_rule_second_block_lower_max():
     v8[129, 0, 3] = 0x38
     cu = np.array([0, n], dtype=np.int32)
     o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True,
-                             rows=[0])
+                             rows=[0], rule=oracle.P_EXP2)
     l = 128 + 2 * math.exp(-0.125)
     assert abs(o[0, 0, 3] - 0.875 / l) < 1e-15
 
@@ -255,14 +255,14 @@ def test_ambiguity_reported_only_at_rounding_ties():
     q8, k8, v8, cu = _two_key_case(0x38)          # k1 = 1.0 * e_0
     ds_k = math.log(29.0 / 32.0)
     o, amb = oracle.attention_fp8(q8, k8, v8, cu, (1.0, ds_k, 1.0), scale=1.0, pquant=True,
-                                  return_ambiguity=True)
+                                  return_ambiguity=True, rule=oracle.P_EXP2)
     l = 1.0 + 29.0 / 32.0
     assert abs(amb[0, 0, 1] - (2.0 / 32.0) / l) < 1e-12
     assert amb[0, 0, 0] == 0.0                    # v1 has no component there
     # y1 = 28.24 (s1 = -0.125) is far from any tie: no allowance
     q8, k8, v8, cu = _two_key_case(0xA0)
     o, amb = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True,
-                                  return_ambiguity=True)
+                                  return_ambiguity=True, rule=oracle.P_EXP2)
     assert (amb == 0.0).all()
 
 
@@ -293,7 +293,7 @@ def test_exp2_tie_window_grows_with_the_accumulation_scale():
     for big, want_amb in ((False, False), (True, True)):
         q8, k8, v8, cu = _two_key_case_with_cancelling_channels(0x38, big)
         o, amb = oracle.attention_fp8(q8, k8, v8, cu, (1.0, ds_k, 1.0), scale=1.0,
-                                      return_ambiguity=True)
+                                      return_ambiguity=True, rule=oracle.P_EXP2)
         assert (amb[0, 0, 1] > 0) == want_amb, (big, amb[0, 0, 1])
         assert abs(o[0, 0, 1] - (30.0 / 32.0) / (1.0 + 29.0 * (1 + 3e-5) / 32.0)) < 1e-12
 
@@ -326,7 +326,7 @@ def test_linear_log_code_interpolates_between_powers_of_two():
     o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, ds_k, 1.0), scale=1.0,
                              rule=oracle.P_LINEAR_LOG)
     assert abs(o[0, 0, 1] - 0.75 / 1.75) < 1e-15
-    e = oracle.attention_fp8(q8, k8, v8, cu, (1.0, ds_k, 1.0), scale=1.0)
+    e = oracle.attention_fp8(q8, k8, v8, cu, (1.0, ds_k, 1.0), scale=1.0, rule=oracle.P_EXP2)
     assert abs(e[0, 0, 1] - 0.6875 / (1.0 + math.sqrt(0.5))) < 1e-15
 
 
