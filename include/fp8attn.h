@@ -324,6 +324,46 @@ fp8attn_status fp8attn_regroup_heads(const void* d_src, void* d_dst, int64_t tok
  * FP8ATTN_ERR_CUDA on a CUDA error.  Takes about 1 s. */
 int fp8attn_selftest_bounded_waits(uint64_t mbar_limit_ns, int* h_gave_up, void* stream);
 
+/* ------------------------------------------------------------------ */
+/* Static scale map (vLLM docs, "FP8 ViT encoder attention": scale file */
+/* format section -- a JSON object mapping each layer name to its      */
+/* {"q", "k", "v"} values, "q_scale"/"k_scale"/"v_scale" accepted as    */
+/* aliases; usage section -- saved values are multiplied by the save    */
+/* margin, 1.5 by default).  Host-only functions, no GPU needed.        */
+/* ------------------------------------------------------------------ */
+
+/* Bytes reserved per layer name in the name arrays below (including the
+ * terminating NUL). */
+#define FP8ATTN_SCALE_NAME_MAX 256
+
+/* h_out[i] = fl32(h_in[i] * margin) for i < n (one fp32 rounding each): the
+ * save margin applied to exported values, or (the other reading of the
+ * page) to stored values when a map is read.  margin must be finite and
+ * > 0; h_in and h_out may be the same array.  Errors: INVALID. */
+fp8attn_status fp8attn_apply_margin(const float* h_in, int64_t n, float margin, float* h_out);
+
+/* Parse a scale map from JSON text (text_len bytes, no NUL needed).  Each
+ * layer's three values are read as doubles, rounded once to fp32 and
+ * multiplied by `margin` (1.0 leaves them as stored); the short key wins
+ * when a layer has both it and its alias; other keys are ignored.  Layers
+ * are returned in file order: names_out [max_layers][FP8ATTN_SCALE_NAME_MAX]
+ * NUL-terminated, values_out [max_layers][3] {q, k, v}; *n_layers_out the
+ * count.  The caller owns every buffer.  Errors: INVALID (malformed JSON, a
+ * missing q/k/v value, a name of FP8ATTN_SCALE_NAME_MAX bytes or more, more
+ * than max_layers layers, a bad margin); *n_layers_out is 0 then. */
+fp8attn_status fp8attn_scale_map_parse(const char* json_text, size_t text_len, float margin,
+                                       int max_layers, char* names_out, float* values_out,
+                                       int* n_layers_out);
+
+/* Write a scale map as JSON text: n_layers names (FP8ATTN_SCALE_NAME_MAX-byte
+ * slots, NUL-terminated) with their {q, k, v} values (finite), each value as
+ * the shortest decimal that reads back as the same fp32 number.  *written
+ * receives the bytes needed including the NUL; if buf is NULL or buf_size is
+ * smaller than that, nothing is written and INVALID is returned (call again
+ * with a larger buffer).  Errors: INVALID. */
+fp8attn_status fp8attn_scale_map_format(int n_layers, const char* names, const float* values,
+                                        char* buf, size_t buf_size, size_t* written);
+
 /* Self-test of the score product (no counterpart in the pages; it checks
  * the accumulation error that the tests' tie model assumes).  For each of
  * `tiles` pairs of 128 x 128 E4M3 tiles -- rows [128 t, 128 t + 128) of

@@ -16,7 +16,6 @@ from __future__ import annotations
 
 import contextlib
 import ctypes
-import json
 import math
 import os
 from typing import Dict, Iterable, List, Optional, Sequence, Tuple
@@ -27,7 +26,7 @@ import torch
 __all__ = [
     "DYNAMIC", "STATIC", "SKIP", "P_LINEAR_LOG", "P_EXP2", "RING_LENGTH", "DEFAULT_MARGIN", "FP8AttnError", "lib",
     "Context", "varlen_fwd", "varlen_fwd_bf16", "parse_selector", "e4m3_encode",
-    "launch_count", "load_scale_file", "save_scale_file", "read_error_word",
+    "launch_count", "load_scale_file", "save_scale_file", "apply_margin", "read_error_word",
     "quantize_qkv_noalloc", "quantize_qkv_noalloc_error", "RING",
     "head_sharded_dynamic_quantize", "regroup_heads", "TorchComm", "ulysses_attention",
 ]
@@ -103,6 +102,11 @@ def lib() -> ctypes.CDLL:
         "fp8attn_selftest_bounded_waits": (I, [ctypes.c_uint64, ctypes.POINTER(I), P]),
         "fp8attn_regroup_heads": (I, [P, P, I64, I, I, I, I, P]),
         "fp8attn_selftest_qk_scores": (I, [P, P, I64, P, P, P]),
+        "fp8attn_apply_margin": (I, [P, I64, F, P]),
+        "fp8attn_scale_map_parse": (I, [ctypes.c_char_p, ctypes.c_size_t, F, I, P, P,
+                                        ctypes.POINTER(I)]),
+        "fp8attn_scale_map_format": (I, [I, P, P, P, ctypes.c_size_t,
+                                         ctypes.POINTER(ctypes.c_size_t)]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -519,42 +523,67 @@ def launch_count() -> int:
     return int(lib().fp8attn_launch_count())
 
 
-_ALIASES = {"q": ("q", "q_scale"), "k": ("k", "k_scale"), "v": ("v", "v_scale")}
+SCALE_NAME_MAX = 256   # FP8ATTN_SCALE_NAME_MAX
+
+
+def apply_margin(values, margin: float = DEFAULT_MARGIN) -> np.ndarray:
+    """fl32(value * margin) for each value (fp8attn_apply_margin): the save
+    margin of the vLLM FP8 ViT page, applied in the library."""
+    v = np.ascontiguousarray(np.asarray(values, dtype=np.float32))
+    out = np.empty_like(v)
+    _check(lib().fp8attn_apply_margin(v.ctypes.data_as(ctypes.c_void_p), v.size,
+                                      float(margin), out.ctypes.data_as(ctypes.c_void_p)),
+           "fp8attn_apply_margin")
+    return out
 
 
 def load_scale_file(path: str, margin: float = 1.0) -> Dict[str, Tuple[float, float, float]]:
     """Read a per-layer {"q","k","v"} scale map (``q_scale``/``k_scale``/
     ``v_scale`` accepted as aliases), as in the vLLM FP8 ViT page's scale
-    file format section.
+    file format section, through fp8attn_scale_map_parse.
 
     The page applies its save margin when the file is written, so by default
     the values are used as stored (``margin=1.0``).  A file written without
     the margin can be read with it applied here: each value becomes
-    fl32(value * margin)."""
-    margin = np.float32(margin)
-    if not np.isfinite(margin) or margin <= 0:
-        raise ValueError("margin must be a positive finite number")
-    with open(path) as f:
-        raw = json.load(f)
+    fl32(value * margin) (in the library)."""
+    with open(path, "rb") as f:
+        text = f.read()
+    cap = max(1, text.count(b":"))          # at least one ':' per layer
+    names = ctypes.create_string_buffer(cap * SCALE_NAME_MAX)
+    values = np.zeros((cap, 3), dtype=np.float32)
+    n = ctypes.c_int(0)
+    status = lib().fp8attn_scale_map_parse(text, len(text), float(margin), cap, names,
+                                           values.ctypes.data_as(ctypes.c_void_p),
+                                           ctypes.byref(n))
+    if status != 0:
+        raise ValueError(f"{path}: not a valid scale map (or margin {margin} not allowed)")
     out = {}
-    for name, entry in raw.items():
-        vals = []
-        for t in ("q", "k", "v"):
-            keys = [k for k in _ALIASES[t] if k in entry]
-            if not keys:
-                raise ValueError(f"layer {name!r} has no {t} value")
-            vals.append(float(np.float32(entry[keys[0]]) * margin))
-        out[name] = tuple(vals)
+    for i in range(n.value):
+        raw = names.raw[i * SCALE_NAME_MAX:(i + 1) * SCALE_NAME_MAX]
+        out[raw[:raw.index(b"\0")].decode()] = tuple(float(x) for x in values[i])
     return out
 
 
 def save_scale_file(path: str, layer_names: Sequence[str], values: np.ndarray) -> None:
-    """Write exported values ([L, 3]) as a per-layer {"q","k","v"} map."""
-    values = np.asarray(values, dtype=np.float32).reshape(len(layer_names), 3)
-    data = {n: {"q": float(v[0]), "k": float(v[1]), "v": float(v[2])}
-            for n, v in zip(layer_names, values)}
-    with open(path, "w") as f:
-        json.dump(data, f, indent=2)
+    """Write exported values ([L, 3]) as a per-layer {"q","k","v"} map
+    (fp8attn_scale_map_format)."""
+    values = np.ascontiguousarray(np.asarray(values, dtype=np.float32).reshape(len(layer_names), 3))
+    names = ctypes.create_string_buffer(max(1, len(layer_names)) * SCALE_NAME_MAX)
+    for i, n in enumerate(layer_names):
+        b = n.encode()
+        if len(b) >= SCALE_NAME_MAX or b"\0" in b:
+            raise ValueError(f"layer name {n!r} too long or holds a NUL")
+        ctypes.memmove(ctypes.addressof(names) + i * SCALE_NAME_MAX, b, len(b))
+    need = ctypes.c_size_t(0)
+    L = lib()
+    L.fp8attn_scale_map_format(len(layer_names), names, values.ctypes.data_as(ctypes.c_void_p),
+                               None, 0, ctypes.byref(need))
+    buf = ctypes.create_string_buffer(need.value)
+    _check(L.fp8attn_scale_map_format(len(layer_names), names,
+                                      values.ctypes.data_as(ctypes.c_void_p), buf, need.value,
+                                      ctypes.byref(need)), "fp8attn_scale_map_format")
+    with open(path, "wb") as f:
+        f.write(buf.value)
 
 
 def selftest_qk_scores(q8: torch.Tensor, k8: torch.Tensor, stream=None) -> torch.Tensor:

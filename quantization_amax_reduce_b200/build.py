@@ -15,7 +15,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["api.cu", "quant.cu", "attention.cu", "regroup.cu"]
+SOURCES = ["api.cu", "quant.cu", "attention.cu", "regroup.cu", "scale_map.cu"]
 HEADERS = ["kernels.h", "sm100_ptx.cuh", "state.cuh"]
 LIB = os.path.join(HERE, "libfp8attn.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

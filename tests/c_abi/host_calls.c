@@ -64,6 +64,32 @@ int main(void) {
                            (const int32_t*)16, 1, 8, 8, 8, 64, (const float*)16, 0.0f,
                            (void*)16, (int32_t*)0, (void*)0) == FP8ATTN_ERR_UNSUPPORTED);
 
+  /* the static scale map: parse (with the margin), format, apply_margin */
+  {
+    static const char text[] =
+        "{\"visual.blocks.0.attn.attn\": {\"q\": 224, \"k\": 198, \"v\": 210},\n"
+        " \"visual.blocks.1.attn.attn\": {\"q_scale\": 218, \"k_scale\": 195, \"v_scale\": 207}}";
+    char names[2 * FP8ATTN_SCALE_NAME_MAX];
+    float vals[6], again[6];
+    int n = -1;
+    size_t need = 0;
+    char out[512];
+    CHECK(fp8attn_scale_map_parse(text, sizeof(text) - 1, 1.0f, 2, names, vals, &n) == FP8ATTN_OK);
+    CHECK(n == 2 && vals[0] == 224.0f && vals[4] == 195.0f);
+    CHECK(strcmp(names + FP8ATTN_SCALE_NAME_MAX, "visual.blocks.1.attn.attn") == 0);
+    CHECK(fp8attn_scale_map_parse(text, sizeof(text) - 1, 1.0f, 1, names, vals, &n) ==
+          FP8ATTN_ERR_INVALID);
+    CHECK(fp8attn_scale_map_parse(text, sizeof(text) - 1, 1.5f, 2, names, vals, &n) == FP8ATTN_OK);
+    CHECK(vals[0] == 336.0f && vals[5] == 310.5f);
+    CHECK(fp8attn_scale_map_format(2, names, vals, (char*)0, 0, &need) == FP8ATTN_ERR_INVALID);
+    CHECK(need > 0 && need <= sizeof(out));
+    CHECK(fp8attn_scale_map_format(2, names, vals, out, sizeof(out), &need) == FP8ATTN_OK);
+    CHECK(fp8attn_scale_map_parse(out, strlen(out), 1.0f, 2, names, again, &n) == FP8ATTN_OK);
+    CHECK(n == 2 && memcmp(vals, again, sizeof(vals)) == 0);
+    CHECK(fp8attn_apply_margin(vals, 6, 1.5f, again) == FP8ATTN_OK && again[0] == 504.0f);
+    CHECK(fp8attn_apply_margin(vals, 6, 0.0f, again) == FP8ATTN_ERR_INVALID);
+  }
+
   if (fails)
     printf("FAILED (%d)\n", fails);
   else

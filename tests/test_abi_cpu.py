@@ -226,3 +226,40 @@ def test_noalloc_sources_checked_before_any_launch(monkeypatch):
     with pytest.raises(ValueError, match="needed"):
         qar.quantize_qkv_noalloc(q, q, q, [0, 100, 128], 100, o, o, o,
                                  torch.zeros(2, dtype=torch.float32))
+
+
+def test_scale_map_parsing_and_margin_in_the_library(tmp_path):
+    """The scale-map reader and writer and the margin multiply are the C
+    library's (fp8attn_scale_map_parse/_format, fp8attn_apply_margin): alias
+    precedence, unknown keys, errors, exact fp32 round trips."""
+    import quantization_amax_reduce_b200 as qar
+    vals = np.array([0.1, 3.0, 1e-3, 448.0, 2.0e38, 224.0, 1.5e-40], dtype=np.float32)
+    want = (vals * np.float32(1.5)).astype(np.float32)
+    np.testing.assert_array_equal(qar.apply_margin(vals, 1.5), want)
+    for bad in (0.0, -2.0, float("inf"), float("nan")):
+        with pytest.raises(qar.FP8AttnError):
+            qar.apply_margin(vals, bad)
+    # the short key wins over its alias; other keys are ignored
+    p = tmp_path / "m.json"
+    p.write_text('{"a": {"q_scale": 9, "q": 1.25, "k": 2, "v_scale": 3.5, "note": [1, {"x": null}]},'
+                 ' "b\\"c": {"q": 0.1, "k": 1e-3, "v": 7}}')
+    m = qar.load_scale_file(str(p))
+    assert m == {"a": (1.25, 2.0, 3.5),
+                 'b"c': (float(np.float32(0.1)), float(np.float32(1e-3)), 7.0)}
+    # errors: malformed text, a missing value, trailing text
+    for text in ('{"a": {"q": 1, "k": 2}}', '{"a": {"q": 1, "k": 2, "v": }}', '{"a": 1}',
+                 '{"a": {"q": 1, "k": 2, "v": 3}} x', '[1, 2]', '{"a": {"q": "1", "k": 2, "v": 3}}'):
+        p.write_text(text)
+        with pytest.raises(ValueError):
+            qar.load_scale_file(str(p))
+    # round trip of awkward values through the writer
+    out = tmp_path / "o.json"
+    names = ["visual.blocks.0.attn", 'with "quote" and \\ slash']
+    arr = np.array([[0.1, 1e-3, 3.0e38], [224.0, 1.5e-40, 0.5]], dtype=np.float32)
+    qar.save_scale_file(str(out), names, arr)
+    back = qar.load_scale_file(str(out))
+    assert list(back) == names
+    for n, row in zip(names, arr):
+        assert back[n] == tuple(float(x) for x in row)
+    # the file is plain JSON that a generic reader accepts too
+    assert set(json.load(open(out))) == set(names)
