@@ -76,7 +76,7 @@ def lib() -> ctypes.CDLL:
     L.or_export_value.argtypes = [ctypes.POINTER(_Ring), f32]
     L.or_attention_fp8.restype = i32
     L.or_attention_fp8.argtypes = [P, P, P, P, i32, i32, i32, f64, f64, f64, f64,
-                                   i32, i32, P, i64, P, P, i32]
+                                   i32, i32, P, i64, P, P, P, P, i32]
     L.or_attention_bf16.restype = i32
     L.or_attention_bf16.argtypes = [P, P, P, P, i32, i32, i32, f64, P, i64, P, i32]
     _lib = L
@@ -229,7 +229,8 @@ P_LINEAR_LOG, P_EXP2 = "linear_log", "exp2"
 
 def attention_fp8(q8, k8, v8, cu, ds_qkv: Sequence[float], scale: Optional[float] = None,
                   pquant: bool = True, l_of_quantized: bool = False, rows=None,
-                  nthreads: int = 0, return_ambiguity: bool = False, rule: str = P_LINEAR_LOG):
+                  nthreads: int = 0, return_ambiguity: bool = False, rule: str = P_LINEAR_LOG,
+                  return_alternative: bool = False):
     """fp64 attention on E4M3 codes [T, H, D]; returns [len(rows) or T, H, D].
 
     With ``pquant`` the PV product uses P quantised per block of 128 keys (in
@@ -252,7 +253,13 @@ def attention_fp8(q8, k8, v8, cu, ds_qkv: Sequence[float], scale: Optional[float
     that P codes lying within an fp32 evaluation's error of a rounding tie
     can make (either neighbouring code is a correct result there), and +inf
     for every output of a row whose reference-max move was decided within
-    such an error of the threshold (that row cannot be compared)."""
+    such an error of the threshold (that row cannot be compared).
+
+    With ``return_alternative`` (implies ``return_ambiguity``) a row whose
+    reference moves exactly once within that error of the threshold is not
+    given up: it is evaluated both ways, and the second result and its
+    allowance come back as two more arrays (NaN for rows with one result);
+    only rows with two or more such decisions keep the infinite allowance."""
     q8 = np.ascontiguousarray(q8, dtype=np.uint8)
     k8 = np.ascontiguousarray(k8, dtype=np.uint8)
     v8 = np.ascontiguousarray(v8, dtype=np.uint8)
@@ -265,12 +272,17 @@ def attention_fp8(q8, k8, v8, cu, ds_qkv: Sequence[float], scale: Optional[float
     r, nr = _rows_arg(rows)
     n = nr if r is not None else int(cu[-1])
     out = np.empty((n, H, D), dtype=np.float64)
+    return_ambiguity = return_ambiguity or return_alternative
     amb = np.empty((n, H, D), dtype=np.float64) if return_ambiguity else None
+    alt = np.empty((n, H, D), dtype=np.float64) if return_alternative else None
+    alt_amb = np.empty((n, H, D), dtype=np.float64) if return_alternative else None
     lib().or_attention_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(cu), cu.size - 1, H, D,
                            float(ds_qkv[0]), float(ds_qkv[1]), float(ds_qkv[2]),
                            float(scale), (2 if rule == P_LINEAR_LOG else 1) if pquant else 0,
                            int(bool(l_of_quantized)),
-                           _ptr(r), nr, _ptr(out), _ptr(amb), nthreads)
+                           _ptr(r), nr, _ptr(out), _ptr(amb), _ptr(alt), _ptr(alt_amb), nthreads)
+    if return_alternative:
+        return out, amb, alt, alt_amb
     return (out, amb) if return_ambiguity else out
 
 

@@ -345,6 +345,8 @@ typedef struct {
     int64_t nrows;
     double* out;              /* [nrows][H][D] */
     double* amb;              /* [nrows][H][D] ambiguity allowance, or NULL */
+    double* alt;              /* [nrows][H][D] the other correct result (NaN: none), or NULL */
+    double* alt_amb;          /* its ambiguity allowance */
     int64_t next;             /* work counter (rows*H items) */
     pthread_mutex_t lock;
 } att_job;
@@ -474,35 +476,21 @@ static double linear_log_ambiguity(double t, double dt) {
     return fabs(or_e4m3_value(hi) - or_e4m3_value(lo)) / OR_P_SCALE;
 }
 
-static void attend_one(const att_job* j, int64_t ri, int h, double* s_buf, double* a_buf) {
-    int64_t t = j->rows ? j->rows[ri] : ri;
-    int b, d;
-    int64_t k0, k1, kk;
-    double M = -INFINITY, l = 0.0, r = -INFINITY, a_r = 0.0, amb_l = 0.0;
-    int unverifiable = 0;
-    double* o = j->out + (ri * j->H + h) * (int64_t)j->D;
-    double* a = j->amb ? j->amb + (ri * j->H + h) * (int64_t)j->D : NULL;
-    double dsq = j->kind == 0 ? j->ds_q : 1.0;
-    double dsk = j->kind == 0 ? j->ds_k : 1.0;
+/* One pass of the P loop over a row's scores (s_buf, a_buf: keys k0..k1-1,
+ * M their max).  The reference r follows the rule; a move decided within
+ * the implementation's error of the threshold is taken as the fp64 test
+ * says, except at block `force_block`, where the opposite is taken.  The
+ * block of the first such decision not forced goes to *first_amb.  Writes
+ * o (and, with a, the tie allowance) already normalised; returns the number
+ * of such decisions not forced. */
+static int attend_pass(const att_job* j, int h, int64_t k0, int64_t k1, const double* s_buf,
+                       const double* a_buf, double M, int64_t force_block, int64_t* first_amb,
+                       double* o, double* a) {
+    int d, n_amb = 0;
+    int64_t kk;
+    double l = 0.0, r = -INFINITY, a_r = 0.0, amb_l = 0.0;
     double dsv = j->kind == 0 ? j->ds_v : 1.0;
-    double sc = dsq * dsk * j->scale;
-    for (b = 0; b < j->B; ++b)
-        if (t >= j->cu[b] && t < j->cu[b + 1]) break;
-    k0 = j->cu[b];
-    k1 = j->cu[b + 1];
-    /* scores: dot of decoded values (exact in fp64 for E4M3), then scales;
-     * A_j = the same sum of absolute products (the error model's scale) */
-    for (kk = k0; kk < k1; ++kk) {
-        double acc = 0.0, aacc = 0.0;
-        for (d = 0; d < j->D; ++d) {
-            double pr = elem(j, j->q, t, h, d) * elem(j, j->k, kk, h, d);
-            acc += pr;
-            aacc += fabs(pr);
-        }
-        s_buf[kk - k0] = acc * sc;
-        a_buf[kk - k0] = aacc * fabs(sc);
-        if (s_buf[kk - k0] > M) M = s_buf[kk - k0];
-    }
+    *first_amb = -1;
     for (d = 0; d < j->D; ++d) o[d] = 0.0;
     if (a)
         for (d = 0; d < j->D; ++d) a[d] = 0.0;
@@ -513,6 +501,7 @@ static void attend_one(const att_job* j, int64_t ri, int h, double* s_buf, doubl
         if ((kk - k0) % OR_P_BLOCK == 0) {
             /* entering a new block: its max, and whether the reference moves */
             int64_t e = kk + OR_P_BLOCK < k1 ? kk + OR_P_BLOCK : k1, x;
+            int64_t blk = (kk - k0) / OR_P_BLOCK;
             double bm = -INFINITY, a_blk = 0.0;
             for (x = kk; x < e; ++x) {
                 if (s_buf[x - k0] > bm) bm = s_buf[x - k0];
@@ -522,8 +511,16 @@ static void attend_one(const att_job* j, int64_t ri, int h, double* s_buf, doubl
                 r = bm;
                 a_r = a_blk;
             } else {
-                if (move_is_ambiguous(bm, a_blk, r, a_r)) unverifiable = 1;
-                if (bm * 1.4426950408889634 > r * 1.4426950408889634 + OR_P_LAG_LOG2) {
+                int move = bm * 1.4426950408889634 > r * 1.4426950408889634 + OR_P_LAG_LOG2;
+                if (move_is_ambiguous(bm, a_blk, r, a_r)) {
+                    if (blk == force_block) {
+                        move = !move;
+                    } else {
+                        if (*first_amb < 0) *first_amb = blk;
+                        ++n_amb;
+                    }
+                }
+                if (move) {
                     r = bm;
                     a_r = a_blk;
                 }
@@ -565,9 +562,60 @@ static void attend_one(const att_job* j, int64_t ri, int h, double* s_buf, doubl
     } else if (a) {
         for (d = 0; d < j->D; ++d) a[d] = a[d] * dsv / l;
     }
-    if (a && unverifiable && j->pquant)
-        for (d = 0; d < j->D; ++d) a[d] = INFINITY;
     for (d = 0; d < j->D; ++d) o[d] = o[d] * dsv / l;
+    return n_amb;
+}
+
+/* One output row (query ri, head h).  When the row's reference moves are all
+ * decided away from the threshold there is one result.  When exactly one is
+ * decided within the implementation's error of it, both outcomes are
+ * correct results of the rule: the row is evaluated both ways and the other
+ * outcome goes to alt / alt_amb (NaN there otherwise).  With more than one
+ * such decision the row is reported as unverifiable (infinite allowance). */
+static void attend_one(const att_job* j, int64_t ri, int h, double* s_buf, double* a_buf,
+                       double* tmp) {
+    int64_t t = j->rows ? j->rows[ri] : ri;
+    int b, d, n_amb;
+    int64_t k0, k1, kk, first_amb, first2;
+    double M = -INFINITY;
+    int64_t base = (ri * j->H + h) * (int64_t)j->D;
+    double* o = j->out + base;
+    double* a = j->amb ? j->amb + base : NULL;
+    double dsq = j->kind == 0 ? j->ds_q : 1.0;
+    double dsk = j->kind == 0 ? j->ds_k : 1.0;
+    double sc = dsq * dsk * j->scale;
+    for (b = 0; b < j->B; ++b)
+        if (t >= j->cu[b] && t < j->cu[b + 1]) break;
+    k0 = j->cu[b];
+    k1 = j->cu[b + 1];
+    /* scores: dot of decoded values (exact in fp64 for E4M3), then scales;
+     * A_j = the same sum of absolute products (the error model's scale) */
+    for (kk = k0; kk < k1; ++kk) {
+        double acc = 0.0, aacc = 0.0;
+        for (d = 0; d < j->D; ++d) {
+            double pr = elem(j, j->q, t, h, d) * elem(j, j->k, kk, h, d);
+            acc += pr;
+            aacc += fabs(pr);
+        }
+        s_buf[kk - k0] = acc * sc;
+        a_buf[kk - k0] = aacc * fabs(sc);
+        if (s_buf[kk - k0] > M) M = s_buf[kk - k0];
+    }
+    n_amb = attend_pass(j, h, k0, k1, s_buf, a_buf, M, -1, &first_amb, o, a);
+    if (j->alt)
+        for (d = 0; d < 2 * j->D; ++d) (d < j->D ? j->alt : j->alt_amb)[base + d % j->D] = NAN;
+    if (!j->pquant || n_amb == 0 || !a) return;
+    if (n_amb == 1 && j->alt) {
+        /* the other outcome of the one decision at the threshold */
+        if (attend_pass(j, h, k0, k1, s_buf, a_buf, M, first_amb, &first2, tmp, tmp + j->D) == 0) {
+            for (d = 0; d < j->D; ++d) {
+                j->alt[base + d] = tmp[d];
+                j->alt_amb[base + d] = tmp[j->D + d];
+            }
+            return;
+        }
+    }
+    for (d = 0; d < j->D; ++d) a[d] = INFINITY;
 }
 
 static void* att_worker(void* arg) {
@@ -577,14 +625,16 @@ static void* att_worker(void* arg) {
     double* s_buf;
     for (b = 0; b < j->B; ++b)
         if (j->cu[b + 1] - j->cu[b] > maxlen) maxlen = j->cu[b + 1] - j->cu[b];
-    s_buf = (double*)malloc(2 * sizeof(double) * (size_t)(maxlen > 0 ? maxlen : 1));
+    s_buf = (double*)malloc(sizeof(double) * (2 * (size_t)(maxlen > 0 ? maxlen : 1) +
+                                              2 * (size_t)j->D));
     for (;;) {
         int64_t w;
         pthread_mutex_lock(&j->lock);
         w = j->next++;
         pthread_mutex_unlock(&j->lock);
         if (w >= total) break;
-        attend_one(j, w / j->H, (int)(w % j->H), s_buf, s_buf + (maxlen > 0 ? maxlen : 1));
+        attend_one(j, w / j->H, (int)(w % j->H), s_buf, s_buf + (maxlen > 0 ? maxlen : 1),
+                   s_buf + 2 * (maxlen > 0 ? maxlen : 1));
     }
     free(s_buf);
     return NULL;
@@ -615,7 +665,7 @@ int or_attention_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
                      const int32_t* cu, int B, int H, int D,
                      double ds_q, double ds_k, double ds_v, double scale,
                      int pquant, int lrule, const int64_t* rows, int64_t nrows,
-                     double* out, double* amb, int nthreads) {
+                     double* out, double* amb, double* alt, double* alt_amb, int nthreads) {
     att_job j;
     memset(&j, 0, sizeof(j));
     j.kind = 0;
@@ -624,6 +674,7 @@ int or_attention_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
     j.ds_q = ds_q; j.ds_k = ds_k; j.ds_v = ds_v; j.scale = scale;
     j.pquant = pquant; j.lrule = lrule;
     j.rows = rows; j.nrows = nrows; j.out = out; j.amb = amb;
+    j.alt = amb ? alt : NULL; j.alt_amb = amb ? alt_amb : NULL;
     return run_attention(&j, nthreads);
 }
 

@@ -39,7 +39,8 @@ def pytest_terminal_summary(terminalreporter, exitstatus, config):
             f"{sum(r['n_excluded'] for r in small)} of {sum(r['n'] for r in small)}")
     for r in rest:
         line = (f"{r['what']}: gated {r['max']:.2e}/{r['mean']:.2e} plain {r['plain_max']:.2e}/"
-                f"{r['plain_mean']:.2e} n={r['n']} tie={r['n_tie']} excl={r['n_excluded']}")
+                f"{r['plain_mean']:.2e} n={r['n']} tie={r['n_tie']} alt={r.get('n_alt', 0)} "
+                f"excl={r['n_excluded']}")
         if r.get("uq"):
             line += f" vs-unquantised {r['uq'][0]:.2e}/{r['uq'][1]:.2e}"
         tr.write_line(line)

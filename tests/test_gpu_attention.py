@@ -54,7 +54,7 @@ def test_fp8_attention_small_shapes(lens, H, rule, orule):
     out = qar.varlen_fwd(q8.to(DEV), k8.to(DEV), v8.to(DEV), torch.as_tensor(cu, device=DEV),
                          max(lens), ds.to(DEV), p_rule=rule)
     want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds.tolist(),
-                                return_ambiguity=True, rule=orule)
+                                return_alternative=True, rule=orule)
     assert_attention_close(out, want, what=f"fp8 {lens} H={H} {orule}")
 
 
@@ -85,7 +85,7 @@ def test_sharp_softmax_rescales(rule, orule):
     ds = [0.25, 0.25, 0.025]
     out = qar.varlen_fwd(q8.to(DEV), k8.to(DEV), v8.to(DEV), torch.as_tensor(cu, device=DEV),
                          900, torch.tensor(ds, device=DEV), p_rule=rule)
-    want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds, return_ambiguity=True,
+    want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds, return_alternative=True,
                                 rule=orule)
     assert_attention_close(out, want, what=f"sharp {orule}")
 
@@ -98,7 +98,7 @@ def test_explicit_softmax_scale(rule, orule):
     out = qar.varlen_fwd(q8.to(DEV), k8.to(DEV), v8.to(DEV), torch.as_tensor(cu, device=DEV),
                          300, torch.tensor(ds, device=DEV), softmax_scale=0.3, p_rule=rule)
     want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds, scale=0.3,
-                                return_ambiguity=True, rule=orule)
+                                return_alternative=True, rule=orule)
     assert_attention_close(out, want, what=f"scale 0.3 {orule}")
 
 
@@ -111,7 +111,7 @@ def test_c1_end_to_end_through_the_boundary(rule, orule):
     out = qar.varlen_fwd(q8, k8, v8, cu_d, 256, ctx.descale_ptr(0), p_rule=rule)
     ol = OracleLayer()
     codes = ol.dynamic_pass([bits(q), bits(k), bits(v)], cu, 2)
-    want = oracle.attention_fp8(*codes, cu, [float(x) for x in ol.ds], return_ambiguity=True,
+    want = oracle.attention_fp8(*codes, cu, [float(x) for x in ol.ds], return_alternative=True,
                                 rule=orule)
     # the error against unquantised fp64 attention on the bf16 inputs is reported
     ref = oracle.attention_bf16(bits(q), bits(k), bits(v), cu)
@@ -138,7 +138,7 @@ def test_c3_full_size_sampled_rows(rule, orule):
     assert_scales_equal(ctx, 0, ol)
     rows = sample_rows(cu, 192, seed=3)
     want = oracle.attention_fp8(*codes, cu, [float(x) for x in ol.ds], rows=rows,
-                                return_ambiguity=True, rule=orule)
+                                return_alternative=True, rule=orule)
     ref = oracle.attention_bf16(hq, hk, hv, cu, rows=rows)
     assert_attention_close(out, want, rows=rows, what=f"c3 {orule}", unquantized=ref)
 
@@ -171,7 +171,7 @@ def test_c2_varlen_after_sixteen_passes_sampled_rows(rule, orule):
     out = qar.varlen_fwd(q8, k8, v8, cu_d, max_len, ctx.descale_ptr(0), p_rule=rule)
     rows = sample_rows(cu, 128, seed=2)
     want = oracle.attention_fp8(*codes, cu, [float(x) for x in ol.ds], rows=rows,
-                                return_ambiguity=True, rule=orule)
+                                return_alternative=True, rule=orule)
     ref = oracle.attention_bf16(hq, hk, hv, cu, rows=rows)
     assert_attention_close(out, want, rows=rows, what=f"c2 {orule}", unquantized=ref)
 
@@ -215,10 +215,10 @@ def test_fp8_nan_in_the_next_sequence_does_not_leak(rule, orule):
     out = qar.varlen_fwd(q8.to(DEV), k8.to(DEV), v8.to(DEV), torch.as_tensor(cu, device=DEV),
                          max(lens), torch.tensor(ds, device=DEV), p_rule=rule)
     want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds,
-                                return_ambiguity=True, rule=orule)
+                                return_alternative=True, rule=orule)
     seq0 = np.arange(cu[0], cu[1])
     assert np.isfinite(out[:cu[1]].float().cpu().numpy()).all()
-    assert_attention_close(out, (want[0][seq0], want[1][seq0]), rows=seq0,
+    assert_attention_close(out, tuple(w[seq0] for w in want), rows=seq0,
                            what=f"fp8 NaN next {orule}")
     assert_attention_close(out, want, what=f"fp8 NaN all {orule}")
 
@@ -267,6 +267,6 @@ def test_reference_max_stays_and_moves_by_design(rule, orule):
     out = qar.varlen_fwd(q8.to(DEV), k8.to(DEV), v8.to(DEV), torch.as_tensor(cu, device=DEV), n,
                          torch.tensor(ds, device=DEV), softmax_scale=1.0, p_rule=rule)
     want = oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), cu, ds, scale=1.0,
-                                return_ambiguity=True, rule=orule)
+                                return_alternative=True, rule=orule)
     assert np.isfinite(want[1]).all()                         # no decision at a tie
     assert_attention_close(out, want, what=f"reference max stays and moves {orule}")

@@ -39,5 +39,5 @@ def test_waits_give_up_at_their_limit_and_the_gpu_stays_usable():
     assert ctx.get_error() == 0
     qs, ds = ctx.get_scales(0)
     want = oracle.attention_fp8(q8.cpu().numpy(), k8.cpu().numpy(), v8.cpu().numpy(), cu,
-                                [float(x) for x in ds], return_ambiguity=True)
+                                [float(x) for x in ds], return_alternative=True)
     assert_attention_close(out, want, what="after the wait probes")

@@ -37,14 +37,14 @@ def test_c4_dit_dynamic_full_size(rule, orule):
     ds = [float(x) for x in ol.ds]
     # every head on a few rows ...
     rows = sample_rows(cu, 24, seed=4)
-    want = oracle.attention_fp8(*codes, cu, ds, rows=rows, return_ambiguity=True, rule=orule)
+    want = oracle.attention_fp8(*codes, cu, ds, rows=rows, return_alternative=True, rule=orule)
     assert_attention_close(out, want, rows=rows, what=f"c4 all heads {orule}")
     # ... and 1024 rows of the first and the last head, with the error
     # against unquantised fp64 attention on the bf16 inputs
     heads = [0, 39]
     rows = sample_rows(cu, 1024, seed=40)
     sub = [np.ascontiguousarray(c[:, heads]) for c in codes]
-    want = oracle.attention_fp8(*sub, cu, ds, rows=rows, return_ambiguity=True, rule=orule)
+    want = oracle.attention_fp8(*sub, cu, ds, rows=rows, return_alternative=True, rule=orule)
     ref = oracle.attention_bf16(*(np.ascontiguousarray(bits(x)[:, heads]) for x in (q, k, v)), cu,
                                 rows=rows)
     assert_attention_close(out[:, heads], want, rows=rows, what=f"c4 1024 rows x 2 heads {orule}",
@@ -125,7 +125,7 @@ def test_c5_calibrate_then_serve():
         out = qar.varlen_fwd(q8, k8, v8, cu_d, max_len, ctx.descale_ptr(l))
         sub = [np.ascontiguousarray(c[:, heads]) for c in codes]
         want = oracle.attention_fp8(*sub, cu, [float(x) for x in ols[l].ds], rows=rows,
-                                    return_ambiguity=True)
+                                    return_alternative=True)
         ref = oracle.attention_bf16(*(np.ascontiguousarray(bits(x)[:, heads]) for x in (q, k, v)),
                                     cu, rows=rows)
         assert_attention_close(out[:, heads], want, rows=rows,

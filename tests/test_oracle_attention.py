@@ -378,3 +378,39 @@ def test_linear_log_rows_average_exactly():
     ones = np.full((T, H, D), 0x38, np.uint8)
     o = oracle.attention_fp8(q8, k8, ones, cu, (0.25, 0.25, 1.0), rule=oracle.P_LINEAR_LOG)
     np.testing.assert_allclose(o, 1.0, rtol=0, atol=1e-13)
+
+
+def test_move_at_the_threshold_gives_two_results_not_an_exclusion():
+    # block 1's max lies 1e-12 above the move threshold (3 ln 2 over r = 0 in
+    # natural units), well inside an implementation's error: with
+    # return_alternative the row comes back evaluated both ways (moved and
+    # not moved), with finite allowances, instead of being given up.  A
+    # second key of block 1 scores 1.0, so the two outcomes quantise it
+    # against references 3 ln 2 + 1e-12 apart.
+    D, n = 128, 130
+    q8 = np.zeros((n, 1, D), np.uint8)
+    k8 = np.zeros((n, 1, D), np.uint8)
+    v8 = np.zeros((n, 1, D), np.uint8)
+    q8[:, 0, 0] = 0x38
+    k8[128, 0, 0] = 0x38                  # s = ds_k (the threshold score)
+    v8[128, 0, 1] = 0x38
+    v8[129, 0, 2] = 0x38
+    v8[0, 0, 3] = 0x38
+    cu = np.array([0, n], dtype=np.int32)
+    ds_k = 3.0 * math.log(2.0) + 1e-12
+    k8[129, 0, 0] = 0x38
+    for rule in (oracle.P_EXP2, oracle.P_LINEAR_LOG):
+        o, amb, alt, alt_amb = oracle.attention_fp8(
+            q8, k8, v8, cu, (1.0, ds_k, 1.0), scale=1.0, rows=[0], rule=rule,
+            return_alternative=True)
+        assert np.isfinite(amb).all() and np.isfinite(alt).all() and np.isfinite(alt_amb).all()
+        np.testing.assert_allclose(alt, o, rtol=0.2, atol=1e-6)
+        # without the alternative the row is reported as unverifiable
+        o2, amb2 = oracle.attention_fp8(q8, k8, v8, cu, (1.0, ds_k, 1.0), scale=1.0, rows=[0],
+                                        rule=rule, return_ambiguity=True)
+        assert np.isinf(amb2).all()
+        np.testing.assert_array_equal(o2, o)
+    # a row whose moves are decided away from the threshold has no alternative
+    o, amb, alt, alt_amb = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0,
+                                                rows=[0], return_alternative=True)
+    assert np.isnan(alt).all() and np.isfinite(amb).all()
