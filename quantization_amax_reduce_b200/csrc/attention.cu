@@ -92,61 +92,6 @@ struct Barriers {
   int abort_flag;
 };
 
-constexpr int kLptMaxBatch = 64;
-
-// The CTA's (sequence b, head h, 256-query block qb).  With several
-// sequences (up to kLptMaxBatch) the units are handed out longest sequence
-// first (ties by index), each sequence's units head by head with the query
-// blocks fastest, so the longest work starts in the first waves and the short
-// sequences fill the tail; CTA indices past the last unit get none (false).
-// A sequence whose cu_seqlens entries are inconsistent gets one unit per
-// head (query block 0) and comes first, so that its CTAs report it.  Called
-// by every thread of the CTA before the warps take their roles.
-__device__ bool decode_unit(const AttnParams& p, int& b, int& h, int& qb) {
-  const int x = blockIdx.x;
-  if (p.B <= 1 || p.B > kLptMaxBatch) {
-    qb = x % p.n_qblk;
-    const int bh = x / p.n_qblk;
-    h = bh % p.H;
-    b = bh / p.H;
-    return true;
-  }
-  __shared__ int s_seq[kLptMaxBatch];     // sequence at each rank
-  __shared__ int s_units[kLptMaxBatch];   // its units (heads x query blocks)
-  auto key_of = [&](int u, int* nq) {
-    const int u0 = __ldg(p.cu + u), u1 = __ldg(p.cu + u + 1), len = u1 - u0;
-    const bool bad = u0 < 0 || len < 0 || len > p.max_seqlen || static_cast<int64_t>(u1) > p.T;
-    if (nq) *nq = bad ? 1 : (len + 255) / 256;
-    return bad ? 0x7FFFFFFF : len;
-  };
-  const int t = threadIdx.x;
-  if (t < p.B) {
-    int nq = 0;
-    const int key = key_of(t, &nq);
-    int rank = 0;
-    for (int u = 0; u < p.B; ++u) {
-      const int ku = key_of(u, nullptr);
-      rank += (ku > key) || (ku == key && u < t);
-    }
-    s_seq[rank] = t;
-    s_units[rank] = nq * p.H;
-  }
-  __syncthreads();
-  int base = 0;
-  for (int r = 0; r < p.B; ++r) {
-    const int n = s_units[r];
-    if (x < base + n) {
-      const int nq = n / p.H;
-      b = s_seq[r];
-      h = (x - base) / nq;
-      qb = (x - base) % nq;
-      return true;
-    }
-    base += n;
-  }
-  return false;
-}
-
 template <typename Bars>
 __device__ __forceinline__ void note_error(AttnParams& p, Bars& bars, uint32_t bit) {
   bars.abort_flag = 1;
@@ -184,8 +129,10 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   const int lane = threadIdx.x & 31;
 
   // ---- work item: (sequence b, head h, query block qb of 256 rows) ----
-  int b, h, qb;
-  if (!decode_unit(p, b, h, qb)) return;
+  const int qb = blockIdx.x % p.n_qblk;
+  const int bh = blockIdx.x / p.n_qblk;
+  const int h = bh % p.H;
+  const int b = bh / p.H;
   const int seq0 = __ldg(p.cu + b);
   const int seq1 = __ldg(p.cu + b + 1);
   const int len = seq1 - seq0;
@@ -573,8 +520,10 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  int b, h, qb;
-  if (!decode_unit(p, b, h, qb)) return;
+  const int qb = blockIdx.x % p.n_qblk;
+  const int bh = blockIdx.x / p.n_qblk;
+  const int h = bh % p.H;
+  const int b = bh / p.H;
   const int seq0 = __ldg(p.cu + b);
   const int seq1 = __ldg(p.cu + b + 1);
   const int len = seq1 - seq0;
