@@ -475,6 +475,36 @@ def measure_per_config(dev, stream, p_rule, fp8_peak, flush):
     res["calibrate_serve_layer3_varlen4_h16"]["seq_lens"] = w.seq_lens(3)
     if ctx.get_error() != 0:
         raise RuntimeError("device error in the per-workload runs")
+
+    # How much of a static-scale step the separate quantisation launch takes
+    # at short and long sequences (the headroom a quantise-in-attention
+    # kernel could recover): one sequence of S tokens, 16 heads, N(0,1),
+    # static 224/198/210, each kernel timed alone after an L2 flush.
+    share = []
+    for S_len in (256, 1024, 4096, 8192):
+        g = torch.Generator(device=dev)
+        g.manual_seed(1000 + S_len)
+        src = [torch.randn(S_len, H, D, generator=g, device=dev).to(torch.bfloat16)
+               for _ in range(3)]
+        cu_s = torch.tensor([0, S_len], dtype=torch.int32, device=dev)
+        cs = qar.Context(1, device=dev)
+        cs.set_static_scales(0, *STATIC)
+        codes = tuple(torch.empty((S_len, H, D), dtype=torch.uint8, device=dev) for _ in range(3))
+        o = torch.empty((S_len, H, D), dtype=torch.bfloat16, device=dev)
+
+        def qz():
+            cs.quantize_qkv(0, qar.STATIC, *src, cu_s, S_len, out=codes, stream=stream)
+
+        def at():
+            qar.varlen_fwd(*codes, cu_s, S_len, cs.descale_ptr(0), out=o, stream=stream,
+                           p_rule=p_rule)
+        qz()
+        at()
+        tq = _time_launches(qz, dev, stream, 20, flush)
+        ta = _time_launches(at, dev, stream, 20, flush)
+        share.append({"S": S_len, "heads": H, "quant_us": tq * 1e6, "attn_us": ta * 1e6,
+                      "quant_share": tq / (tq + ta)})
+    res["static_quant_share_by_length"] = share
     return res
 
 
