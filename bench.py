@@ -390,13 +390,29 @@ def _unquantized_reference(q, k, v, cu, rows, heads):
     return out
 
 
-def _err_vs_unquantized(out, q, k, v, cu, rows, heads):
+def _err_vs_unquantized(out, q, k, v, cu, rows, heads, codes=None, descales=None):
+    """Error of the FP8 output against fp64 attention on the bf16 inputs on
+    sampled rows, with the output's RMS for scale.  Given the E4M3 codes and
+    their descales it also reports ``inputs_only``: the same error for fp64
+    attention on the dequantised codes, i.e. what input quantisation alone
+    costs before any P rounding (peaked attention, as in the low-rank Q/K
+    workload, turns small score errors into O(1) output differences)."""
     import torch
-    ref = _unquantized_reference(q.cpu(), k.cpu(), v.cpu(), cu, rows, heads)
+    sel = list(range(len(heads)))
+    hi = torch.as_tensor(heads, device=q.device)
+    ref = _unquantized_reference(*(x.index_select(1, hi).cpu() for x in (q, k, v)), cu, rows, sel)
     got = out.cpu()[rows][:, heads].double()
     d = (got - ref).abs()
-    return {"max": float(d.max()), "mean": float(d.mean()), "rows": len(rows),
-            "heads": list(heads)}
+    res = {"max": float(d.max()), "mean": float(d.mean()),
+           "ref_rms": float(ref.pow(2).mean().sqrt()), "rows": len(rows),
+           "heads": list(heads)}
+    if codes is not None:
+        deq = [c.index_select(1, hi).cpu().view(torch.float8_e4m3fn).double() * float(s)
+               for c, s in zip(codes, descales)]
+        ref_q = _unquantized_reference(*deq, cu, rows, sel)
+        dq = (ref_q - ref).abs()
+        res["inputs_only"] = {"max": float(dq.max()), "mean": float(dq.mean())}
+    return res
 
 
 def _sample_rows(cu, per_seq, seed):
@@ -424,7 +440,7 @@ def measure_per_config(dev, stream, p_rule, fp8_peak, flush):
     res = {}
 
     def attn_entry(name, q8, k8, v8, cu, cu_d, max_len, ds_ptr, flops, q, k, v, rows, heads,
-                   reps):
+                   reps, descales):
         T, Hn = q8.shape[0], q8.shape[1]
         out = torch.empty((T, Hn, D), dtype=torch.bfloat16, device=dev)
 
@@ -436,7 +452,7 @@ def measure_per_config(dev, stream, p_rule, fp8_peak, flush):
         tf = flops / sec / 1e12
         res[name] = {"attn_us": sec * 1e6, "attn_tflops": tf, "frac": tf / fp8_peak,
                      "flops": flops, "err_vs_unquantized": _err_vs_unquantized(
-                         out, q, k, v, cu, rows, heads)}
+                         out, q, k, v, cu, rows, heads, (q8, k8, v8), descales)}
 
     # config 2: ViT-shaped varlen batch after its 16 dynamic passes
     w = synthetic.WORKLOADS[2]
@@ -448,7 +464,8 @@ def measure_per_config(dev, stream, p_rule, fp8_peak, flush):
         q, k, v, _ = synthetic.qkv(2, 0, p, device=dev)
         q8, k8, v8 = ctx.quantize_qkv(0, qar.DYNAMIC, q, k, v, cu_d, max_len, stream=stream)
     attn_entry("vit_varlen3_h16_after_16_passes", q8, k8, v8, cu, cu_d, max_len,
-               ctx.descale_ptr(0), w.flops(0), q, k, v, _sample_rows(cu, 6, 2), [0, 15], 10)
+               ctx.descale_ptr(0), w.flops(0), q, k, v, _sample_rows(cu, 6, 2), [0, 15], 10,
+               ctx.get_scales(0, stream=stream)[1])
     res["vit_varlen3_h16_after_16_passes"]["seq_lens"] = w.seq_lens(0)
     del q, k, v, q8, k8, v8
 
@@ -459,7 +476,8 @@ def measure_per_config(dev, stream, p_rule, fp8_peak, flush):
     ctx = qar.Context(1, device=dev)
     q8, k8, v8 = ctx.quantize_qkv(0, qar.DYNAMIC, q, k, v, cu_d, 32760, stream=stream)
     attn_entry("dit_s32760_h40_dynamic", q8, k8, v8, cu, cu_d, 32760, ctx.descale_ptr(0),
-               w.flops(0), q, k, v, _sample_rows(cu, 8, 4), [0, 39], 5)
+               w.flops(0), q, k, v, _sample_rows(cu, 8, 4), [0, 39], 5,
+               ctx.get_scales(0, stream=stream)[1])
     del q, k, v, q8, k8, v8
 
     # config 5: one served layer (layer 3 of 24, dynamic pass on its inputs)
@@ -471,7 +489,8 @@ def measure_per_config(dev, stream, p_rule, fp8_peak, flush):
     ctx = qar.Context(1, device=dev)
     q8, k8, v8 = ctx.quantize_qkv(0, qar.DYNAMIC, q, k, v, cu_d, max_len, stream=stream)
     attn_entry("calibrate_serve_layer3_varlen4_h16", q8, k8, v8, cu, cu_d, max_len,
-               ctx.descale_ptr(0), w.flops(3), q, k, v, _sample_rows(cu, 4, 5), [0, 15], 5)
+               ctx.descale_ptr(0), w.flops(3), q, k, v, _sample_rows(cu, 4, 5), [0, 15], 5,
+               ctx.get_scales(0, stream=stream)[1])
     res["calibrate_serve_layer3_varlen4_h16"]["seq_lens"] = w.seq_lens(3)
     if ctx.get_error() != 0:
         raise RuntimeError("device error in the per-workload runs")
@@ -790,7 +809,8 @@ def run_ours(args):
 
     # this workload's error against unquantised fp64 attention, and the
     # attention time under the other P rule (outside the timed step)
-    err_uq = _err_vs_unquantized(out, q, k, v, cu, _sample_rows(cu, 24, 3), list(range(H)))
+    err_uq = _err_vs_unquantized(out, q, k, v, cu, _sample_rows(cu, 24, 3), list(range(H)),
+                                 (q8, k8, v8), ctx.get_scales(0, stream=stream)[1])
     other = "exp2" if args.p_rule == "linear_log" else "linear_log"
 
     def attn_other():

@@ -111,7 +111,8 @@ def sample_rows(cu: np.ndarray, per_seq: int, seed: int = 0) -> np.ndarray:
 def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
     """Half the spacing of bf16 numbers at |x| (bf16 keeps 8 significant
     bits: spacing 2^(e-7) in [2^e, 2^(e+1)); subnormal spacing below 2^-126)."""
-    a = np.maximum(np.abs(np.asarray(x, dtype=np.float64)), 2.0 ** -126)
+    a = np.abs(np.asarray(x, dtype=np.float64))
+    a = np.where(np.isfinite(a), np.maximum(a, 2.0 ** -126), 2.0 ** 127)   # non-finite: any
     e = np.floor(np.log2(a))
     return np.ldexp(1.0, (e - 8).astype(np.int64))
 
