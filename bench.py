@@ -818,6 +818,14 @@ def run_ours(args):
                        p_rule=P_RULES[other])
     attn_other()
     other_s = _time_launches(attn_other, dev, stream, 20, flush_l2)
+
+    # the same attention with one CTA per work unit (the timed step uses the
+    # automatic schedule, which splits the units of a mostly empty last wave)
+    def attn_whole():
+        qar.varlen_fwd(q8, k8, v8, cu_d, S, ds_ptr, out=out, stream=stream,
+                       p_rule=P_RULES[args.p_rule], schedule=qar.SCHED_WHOLE)
+    attn_whole()
+    whole_s = _time_launches(attn_whole, dev, stream, 20, flush_l2)
     per_config = None
     if world == 1 and not args.no_per_config:
         per_config = measure_per_config(dev, stream, p_rule, fp8_peak, flush_l2)
@@ -847,6 +855,8 @@ def run_ours(args):
             "attn_us": attn_s * 1e6, "attn_tflops": attn_tflops,
             "attn_other_rule": {"p_rule": other, "attn_us": other_s * 1e6,
                                 "attn_tflops": FLOPS_PER_STEP / other_s / 1e12},
+            "attn_whole_units": {"schedule": "one CTA per unit", "attn_us": whole_s * 1e6,
+                                 "attn_tflops": FLOPS_PER_STEP / whole_s / 1e12},
             "err_vs_unquantized": err_uq,
             "quant_us": quant_s * 1e6, "quant_gbs": quant_gbs,
             "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": fp8_peak,

@@ -36,6 +36,8 @@ LIB_PATH = os.path.join(HERE, "libfp8attn.so")
 
 DYNAMIC, STATIC, SKIP, RING = 0, 1, 2, 3
 P_LINEAR_LOG, P_EXP2 = 0, 1
+# work schedules of the FP8 attention kernel (fp8attn_schedule in fp8attn.h)
+SCHED_AUTO, SCHED_WHOLE, SCHED_SPLIT = 0, 1, 2
 RING_LENGTH = 16
 DEFAULT_MARGIN = 1.5
 HEAD_DIM = 128
@@ -88,6 +90,7 @@ def lib() -> ctypes.CDLL:
         "fp8attn_get_scales": (I, [P, I, P, P]),
         "fp8attn_varlen_fwd": (I, [P, P, P, P, I, I, I64, I, I, P, F, P, P, P]),
         "fp8attn_varlen_fwd_rule": (I, [P, P, P, P, I, I, I64, I, I, P, F, I, P, P, P]),
+        "fp8attn_varlen_fwd_sched": (I, [P, P, P, P, I, I, I64, I, I, P, F, I, I, P, P, P]),
         "fp8attn_varlen_fwd_bf16": (I, [P, P, P, P, I, I, I64, I, I, F, P, P, P]),
         "fp8attn_get_error": (I, [P, P]),
         "fp8attn_read_error_word": (I, [P, P]),
@@ -411,12 +414,15 @@ def _attn_common(q, k, v, cu_seqlens, out, dtype):
 def varlen_fwd(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, cu_seqlens,
                max_seqlen: int, descale, softmax_scale: float = 0.0,
                out: Optional[torch.Tensor] = None, error: Optional[torch.Tensor] = None,
-               stream=None, p_rule: int = P_LINEAR_LOG) -> torch.Tensor:
+               stream=None, p_rule: int = P_LINEAR_LOG,
+               schedule: int = SCHED_AUTO) -> torch.Tensor:
     """FP8 attention on packed E4M3 [T, H, 128] codes.  ``descale`` is a device
     pointer (int, e.g. ``Context.descale_ptr(layer)``) or a 3-element fp32 CUDA
     tensor {ds_q, ds_k, ds_v}.  ``p_rule`` picks how P is quantised for the PV
     product (P_LINEAR_LOG, the default, or P_EXP2; see fp8attn_p_rule in
-    fp8attn.h).
+    fp8attn.h); ``schedule`` how the work units are laid on the GPU
+    (SCHED_AUTO, SCHED_WHOLE or SCHED_SPLIT; the same result up to fp32
+    rounding, see fp8attn_schedule).
     Returns bf16 [T, H, 128]."""
     T, H, cu, out = _attn_common(q8, k8, v8, cu_seqlens, out, torch.uint8)
     if isinstance(descale, torch.Tensor):
@@ -426,11 +432,12 @@ def varlen_fwd(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, cu_seqlens,
         dptr = ctypes.c_void_p(descale.data_ptr())
     else:
         dptr = ctypes.c_void_p(int(descale))
-    _check(lib().fp8attn_varlen_fwd_rule(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(cu), cu.numel() - 1,
-                                         int(max_seqlen), T, H, HEAD_DIM, dptr,
-                                         float(softmax_scale), int(p_rule), _ptr(out),
-                                         _ptr(error), ctypes.c_void_p(_stream(stream, q8.device))),
-           "fp8attn_varlen_fwd_rule")
+    _check(lib().fp8attn_varlen_fwd_sched(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(cu), cu.numel() - 1,
+                                          int(max_seqlen), T, H, HEAD_DIM, dptr,
+                                          float(softmax_scale), int(p_rule), int(schedule),
+                                          _ptr(out), _ptr(error),
+                                          ctypes.c_void_p(_stream(stream, q8.device))),
+           "fp8attn_varlen_fwd_sched")
     return out
 
 

@@ -71,8 +71,12 @@ fp8attn_status check_attention(const void* q, const void* k, const void* v,
 fp8attn_status run_attention(const void* q, const void* k, const void* v, const int32_t* cu,
                              int batch, int max_seqlen, int64_t total_tokens, int num_heads,
                              int head_dim, const float* descale, float softmax_scale, void* out,
-                             int32_t* err, void* stream, int bf16, int p_rule) {
+                             int32_t* err, void* stream, int bf16, int p_rule,
+                             int schedule) {
   if (p_rule != FP8ATTN_P_LINEAR_LOG && p_rule != FP8ATTN_P_EXP2) return FP8ATTN_ERR_INVALID;
+  if (schedule != FP8ATTN_SCHED_AUTO && schedule != FP8ATTN_SCHED_WHOLE &&
+      schedule != FP8ATTN_SCHED_SPLIT)
+    return FP8ATTN_ERR_INVALID;
   fp8attn_status st = check_attention(q, k, v, cu, batch, max_seqlen, total_tokens, num_heads,
                                       head_dim, out);
   if (st != FP8ATTN_OK || total_tokens == 0) return st;
@@ -93,6 +97,9 @@ fp8attn_status run_attention(const void* q, const void* k, const void* v, const 
   a.err = err;
   a.bf16 = bf16;
   a.p_rule = p_rule == FP8ATTN_P_EXP2 ? kPRuleExp2 : kPRuleLinearLog;
+  a.schedule = schedule == FP8ATTN_SCHED_WHOLE   ? kSchedWhole
+               : schedule == FP8ATTN_SCHED_SPLIT ? kSchedSplit
+                                                 : kSchedAuto;
   const cudaError_t e = launch_attention(a, total_tokens, as_stream(stream));
   if (e != cudaSuccess) return FP8ATTN_ERR_CUDA;
   g_launches.fetch_add(1);
@@ -377,7 +384,7 @@ fp8attn_status fp8attn_varlen_fwd(const void* q8, const void* k8, const void* v8
                                   int32_t* d_error, void* stream) {
   return run_attention(q8, k8, v8, d_cu_seqlens, batch, max_seqlen, total_tokens, num_heads,
                        head_dim, d_descale_qkv, softmax_scale, out, d_error, stream, 0,
-                       FP8ATTN_P_LINEAR_LOG);
+                       FP8ATTN_P_LINEAR_LOG, FP8ATTN_SCHED_AUTO);
 }
 
 fp8attn_status fp8attn_varlen_fwd_rule(const void* q8, const void* k8, const void* v8,
@@ -386,7 +393,19 @@ fp8attn_status fp8attn_varlen_fwd_rule(const void* q8, const void* k8, const voi
                                        const float* d_descale_qkv, float softmax_scale,
                                        int p_rule, void* out, int32_t* d_error, void* stream) {
   return run_attention(q8, k8, v8, d_cu_seqlens, batch, max_seqlen, total_tokens, num_heads,
-                       head_dim, d_descale_qkv, softmax_scale, out, d_error, stream, 0, p_rule);
+                       head_dim, d_descale_qkv, softmax_scale, out, d_error, stream, 0, p_rule,
+                       FP8ATTN_SCHED_AUTO);
+}
+
+fp8attn_status fp8attn_varlen_fwd_sched(const void* q8, const void* k8, const void* v8,
+                                        const int32_t* d_cu_seqlens, int batch, int max_seqlen,
+                                        int64_t total_tokens, int num_heads, int head_dim,
+                                        const float* d_descale_qkv, float softmax_scale,
+                                        int p_rule, int schedule, void* out, int32_t* d_error,
+                                        void* stream) {
+  return run_attention(q8, k8, v8, d_cu_seqlens, batch, max_seqlen, total_tokens, num_heads,
+                       head_dim, d_descale_qkv, softmax_scale, out, d_error, stream, 0, p_rule,
+                       schedule);
 }
 
 fp8attn_status fp8attn_selftest_qk_scores(const void* d_q8, const void* d_k8, int64_t tiles,
@@ -409,7 +428,7 @@ fp8attn_status fp8attn_varlen_fwd_bf16(const void* q, const void* k, const void*
                                        void* stream) {
   return run_attention(q, k, v, d_cu_seqlens, batch, max_seqlen, total_tokens, num_heads,
                        head_dim, nullptr, softmax_scale, out, d_error, stream, 1,
-                       FP8ATTN_P_EXP2);
+                       FP8ATTN_P_EXP2, FP8ATTN_SCHED_WHOLE);
 }
 
 fp8attn_status fp8attn_get_error(fp8attn_ctx* ctx, void* stream) {

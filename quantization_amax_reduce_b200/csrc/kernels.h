@@ -46,11 +46,17 @@ struct AttnLaunch {
   int32_t* err;                  // device error word or null
   int bf16;                      // 1 = native bf16 inputs (skip-layer path)
   int p_rule;                    // FP8 only: kPRuleLinearLog or kPRuleExp2
+  int schedule;                  // FP8 only: kSchedAuto, kSchedWhole or kSchedSplit
 };
 
 // P rules of the FP8 kernel (the values of fp8attn_p_rule in fp8attn.h).
 constexpr int kPRuleLinearLog = 0;
 constexpr int kPRuleExp2 = 1;
+
+// Work schedules of the FP8 kernel (the values of fp8attn_schedule).
+constexpr int kSchedAuto = 0;    // split the units of a last wave at most half full
+constexpr int kSchedWhole = 1;   // one CTA per unit
+constexpr int kSchedSplit = 2;   // every unit long enough as a pair of CTAs
 
 cudaError_t launch_attention(const AttnLaunch& p, int64_t total_tokens, cudaStream_t stream);
 

@@ -93,6 +93,11 @@ def test_host_argument_checks_need_no_gpu(L):
     # zero tokens is a no-op
     assert L.fp8attn_varlen_fwd(None, None, None, P(16), 1, 8, 0, 8, 128, None, 0.0, None,
                                 None, None) == 0
+    # an unknown P rule or work schedule is invalid; the known ones pass the
+    # checks (zero tokens: nothing launched)
+    for rule, sched, want in ((0, 3, 1), (0, -1, 1), (2, 0, 1), (1, 2, 0), (0, 1, 0)):
+        assert L.fp8attn_varlen_fwd_sched(None, None, None, P(16), 1, 8, 0, 8, 128, None, 0.0,
+                                          rule, sched, None, None, None) == want
     assert L.fp8attn_create(0, P(256), 1 << 20, None, ctypes.byref(P())) == 1
     assert L.fp8attn_e4m3_encode(None, 5, 1.0, None, None) == 1
     # the amax-only entry point rejects a null context, a null output, a bad
