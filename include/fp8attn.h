@@ -220,9 +220,7 @@ fp8attn_status fp8attn_varlen_fwd(const void* q8, const void* k8, const void* v8
  * PV product (the pages give none; both are defined in full here).  With
  * c = ds_q ds_k softmax_scale log2(e), a per-row reference m (log2 units; the
  * first 128-key block's max of s c, moved to a later block's max only when
- * that exceeds m by more than 3, and set afresh to the block's max at the
- * first block of every 4096-key segment of the sequence) and
- * t = s c - m + 5 <= 8:
+ * that exceeds m by more than 3) and t = s c - m + 5 <= 8:
  *   FP8ATTN_P_LINEAR_LOG: code = RNE(8 t + 56) clamped to [0, 128] -- the
  *     E4M3 bit pattern read as a fixed-point log2 (Mitchell's / Schraudolph's
  *     piecewise-linear 2^t, exponent and mantissa filled linearly from t);
@@ -230,28 +228,23 @@ fp8attn_status fp8attn_varlen_fwd(const void* q8, const void* k8, const void* v8
  *     adds the E4M3 values of the codes.
  *   FP8ATTN_P_EXP2: code = e4m3_rne(2^t) (2^t evaluated to about 2^-22
  *     relative); l adds the unquantised 2^t.
- * Both: out = (sum_j P_j v_j) ds_v / l, with every P_j carried to one scale
- * by 2^(m_j - M) (m_j the reference its block used, M the row's largest).
- * Because of the segment restart, a row may be evaluated as separate key
- * ranges split at segment boundaries and combined with the same result up to
- * fp32 rounding.  (The kernel leaves out a block whose reference lies more
- * than 2^64 below the scale of the blocks before it: weights below 2^-61.) */
+ * Both: out = (sum_j P_j v_j) ds_v / l, with P carried across moves of m by
+ * 2^(m_old - m_new). */
 typedef enum {
   FP8ATTN_P_LINEAR_LOG = 0,
   FP8ATTN_P_EXP2 = 1
 } fp8attn_p_rule;
 
 /* How fp8attn_varlen_fwd_sched lays the work units (256 query rows of one
- * head of one sequence) on the GPU.  The result is the same under every
- * schedule up to fp32 rounding (see the segment restart above).
+ * head of one sequence, computed as two 128-row tiles) on the GPU.  Each
+ * output row is computed the same way under every schedule (same key
+ * blocks, order and P rule), so the results are bit-identical.
  *   FP8ATTN_SCHED_AUTO: one CTA per unit, except that when the last wave of
- *     units would fill at most half of the SMs, those units each run on a
- *     cluster of two CTAs that take the two sides of the 4096-key segment
- *     boundary nearest the middle of the row and combine their halves of the
- *     output through distributed shared memory (a second launch).
+ *     units would fill at most half of the SMs, each of those units runs as
+ *     two CTAs of one tile each, so that the tiles fill that wave (a lone
+ *     tile's blocks run faster than a CTA's two interleaved tiles).
  *   FP8ATTN_SCHED_WHOLE: one CTA per unit.
- *   FP8ATTN_SCHED_SPLIT: every unit as a CTA pair (units of sequences no
- *     longer than 4096 keys run whole in the pair's first CTA). */
+ *   FP8ATTN_SCHED_SPLIT: every unit as two single-tile CTAs. */
 typedef enum {
   FP8ATTN_SCHED_AUTO = 0,
   FP8ATTN_SCHED_WHOLE = 1,

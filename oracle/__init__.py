@@ -236,9 +236,8 @@ def attention_fp8(q8, k8, v8, cu, ds_qkv: Sequence[float], scale: Optional[float
     With ``pquant`` the PV product uses P quantised per block of 128 keys (in
     sequence order) as e4m3(32 exp(s - r))/32 against the row's reference max
     r: block 0's max, replaced by a later block's max only when that exceeds
-    r by more than 3 in log2 units, and started afresh (as at block 0) at the
-    first block of every 4096-key segment; each block is carried exactly to
-    the final max M; l is the sum of the unquantised exp(s - M) unless
+    r by more than 3 in log2 units; each block is carried exactly to the final
+    max M; l is the sum of the unquantised exp(s - M) unless
     ``l_of_quantized``.
 
     ``rule`` selects the quantisation of each block's P (both against the

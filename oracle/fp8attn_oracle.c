@@ -362,17 +362,10 @@ static double elem(const att_job* j, const void* base, int64_t t, int h, int d) 
  * e4m3(OR_P_SCALE exp(s - r_t)) / OR_P_SCALE against the row's reference max
  * r_t, then carried to the final max M by the exact factor exp(r_t - M).
  * r_0 is block 0's max; r_t is block t's max when that exceeds r_{t-1} by
- * more than OR_P_LAG_LOG2 in log2 units, else r_{t-1}.  The reference starts
- * afresh at every segment of OR_P_SEGMENT_BLOCKS blocks (keys 4096 n, n >= 1,
- * from the start of the sequence): there r_t is block t's max, as at the
- * first block, so a row's segments can be evaluated apart and combined (the
- * exact factor exp(r_t - M) already places every block on one scale).  A
- * block whose keys are all NaN or masked has max -inf and leaves the
- * reference at -inf, so the next block starts it.  With the lag at most 3 and
- * the scale 2^5, OR_P_SCALE exp(s - r_t) <= 2^8 (no saturation).  l is the
- * sum of the unquantised p = exp(s - M). */
+ * more than OR_P_LAG_LOG2 in log2 units, else r_{t-1}.  With the lag at most
+ * 3 and the scale 2^5, OR_P_SCALE exp(s - r_t) <= 2^8 (no saturation).  l is
+ * the sum of the unquantised p = exp(s - M). */
 #define OR_P_BLOCK 128
-#define OR_P_SEGMENT_BLOCKS 32
 #define OR_P_SCALE 32.0
 #define OR_P_LAG_LOG2 3.0
 
@@ -514,8 +507,7 @@ static int attend_pass(const att_job* j, int h, int64_t k0, int64_t k1, const do
                 if (s_buf[x - k0] > bm) bm = s_buf[x - k0];
                 if (a_buf[x - k0] > a_blk) a_blk = a_buf[x - k0];
             }
-            if (r == -INFINITY || blk % OR_P_SEGMENT_BLOCKS == 0) {
-                /* first block of the row or of a segment: the reference starts here */
+            if (r == -INFINITY) {
                 r = bm;
                 a_r = a_blk;
             } else {

@@ -421,8 +421,8 @@ def varlen_fwd(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, cu_seqlens,
     tensor {ds_q, ds_k, ds_v}.  ``p_rule`` picks how P is quantised for the PV
     product (P_LINEAR_LOG, the default, or P_EXP2; see fp8attn_p_rule in
     fp8attn.h); ``schedule`` how the work units are laid on the GPU
-    (SCHED_AUTO, SCHED_WHOLE or SCHED_SPLIT; the same result up to fp32
-    rounding, see fp8attn_schedule).
+    (SCHED_AUTO, SCHED_WHOLE or SCHED_SPLIT; bit-identical results, see
+    fp8attn_schedule).
     Returns bf16 [T, H, 128]."""
     T, H, cu, out = _attn_common(q8, k8, v8, cu_seqlens, out, torch.uint8)
     if isinstance(descale, torch.Tensor):
@@ -726,7 +726,8 @@ def _single_seq_cu(S: int, device) -> torch.Tensor:
 
 def ulysses_attention(ctx: "Context", layer: int, mode: int, q: torch.Tensor, k: torch.Tensor,
                       v: torch.Tensor, comm=None, softmax_scale: float = 0.0,
-                      stream=None, p_rule: int = P_LINEAR_LOG) -> torch.Tensor:
+                      stream=None, p_rule: int = P_LINEAR_LOG,
+                      schedule: int = SCHED_AUTO) -> torch.Tensor:
     """Sequence-parallel (Ulysses) attention over one sequence whose tokens are
     split evenly across the ranks of ``comm`` (a :class:`TorchComm` by
     default): rank r holds tokens [r S_loc, (r+1) S_loc) of Q, K, V as bf16
@@ -744,8 +745,9 @@ def ulysses_attention(ctx: "Context", layer: int, mode: int, q: torch.Tensor, k:
     on those heads, the return all-to-all, and the inverse head regrouping.
     SKIP regroups and exchanges bf16 and runs the bf16 attention.  Codes,
     scales, ring and output equal one single-GPU pass over the whole sequence
-    (``quantize_qkv`` with the same mode, then ``varlen_fwd``).  Every rank
-    must make the same calls in the same order."""
+    (``quantize_qkv`` with the same mode, then ``varlen_fwd``), bit for bit
+    under any work ``schedule``.  Every rank must make the same calls in the
+    same order."""
     comm = TorchComm() if comm is None else comm
     n = int(comm.size())
     if q.dim() != 3 or q.shape != k.shape or q.shape != v.shape:
@@ -792,7 +794,7 @@ def ulysses_attention(ctx: "Context", layer: int, mode: int, q: torch.Tensor, k:
             o = varlen_fwd_bf16(recv[0], recv[1], recv[2], cu_all, S, softmax_scale)
         else:
             o = varlen_fwd(recv[0], recv[1], recv[2], cu_all, S, ctx.descale_ptr(layer),
-                           softmax_scale, p_rule=p_rule)
+                           softmax_scale, p_rule=p_rule, schedule=schedule)
         if n == 1:
             return o.view(S_loc, H, D)
         back = torch.empty_like(o)

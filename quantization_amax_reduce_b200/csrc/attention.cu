@@ -56,15 +56,6 @@ constexpr int kPolyEvery = 4;
 // P = e4m3(2^(t - r + kPOffsetLog2)) stays at or below 2^(kRefLag + kPOffsetLog2) = 256.
 constexpr float kRefLag = 3.0f;
 constexpr float kPOffsetLog2 = 5.0f;
-// FP8 P rule: the reference restarts at the first block of every segment of
-// kSegBlocks 128-key blocks (4096 keys), so a row's key range can be split
-// at a segment boundary and the two sides combined on one scale.
-constexpr int kSegBlocks = 32;
-// FP8 kernel: the scale of O and l follows the reference down (at a segment
-// restart) by at most 2^kMaxDrop; a block whose reference lies further below
-// contributes weights under 2^-(kMaxDrop - 3) of the row's largest and is
-// dropped, which keeps every rescale factor below 2^64 (no fp32 overflow).
-constexpr float kMaxDrop = 64.0f;
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -81,8 +72,10 @@ struct Bf16Cfg {
 struct AttnParams {
   const int32_t* cu;
   int B, H, max_seqlen, n_qblk;   // n_qblk = query blocks of 256 rows per sequence
-  int unit0;                      // first work unit (query block, head, sequence) of the launch
-  int split;                      // FP8: 1 = each unit runs as a pair of CTAs (cluster of 2)
+  // FP8: CTAs [0, n_whole) each run one work unit (256 query rows of one
+  // head) as two 128-row tiles; every CTA after them runs one tile of the
+  // units from n_whole on (two CTAs per unit)
+  int n_whole;
   int64_t T;
   const float* descale;
   float softmax_scale;
@@ -531,10 +524,12 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // work unit = (query block of 256 rows, head, sequence); in a split launch
-  // CTAs 2u and 2u + 1 (one cluster) share unit u
-  const int unit = p.unit0 + static_cast<int>(p.split ? blockIdx.x >> 1 : blockIdx.x);
-  const int half = p.split ? static_cast<int>(cluster_ctarank()) : 0;
+  // work unit = (query block of 256 rows, head, sequence); a CTA past
+  // n_whole takes one 128-row half of a unit (ntiles = 1)
+  const int cta = static_cast<int>(blockIdx.x);
+  const int ntiles = cta < p.n_whole ? 2 : 1;
+  const int unit = cta < p.n_whole ? cta : p.n_whole + ((cta - p.n_whole) >> 1);
+  const int sub = cta < p.n_whole ? 0 : ((cta - p.n_whole) & 1);
   const int qb = unit % p.n_qblk;
   const int bh = unit / p.n_qblk;
   const int h = bh % p.H;
@@ -543,46 +538,21 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int seq1 = __ldg(p.cu + b + 1);
   const int len = seq1 - seq0;
   if (seq0 < 0 || len < 0 || len > p.max_seqlen || static_cast<int64_t>(seq1) > p.T) {
-    if (threadIdx.x == 0 && qb == 0 && half == 0 && p.err)
+    if (threadIdx.x == 0 && qb == 0 && sub == 0 && p.err)
       atomicOr(reinterpret_cast<unsigned int*>(p.err), kErrSeqlens);
     return;
   }
-  const int q0 = qb * 256;
+  const int q0 = qb * 256 + 128 * sub;   // first query row of this CTA's tile 0
   if (q0 >= len) return;
-  const int nblk = (len + 127) / 128;
-  // key blocks [kb0, kb1) of this CTA: the two CTAs of a pair take the two
-  // sides of the segment boundary nearest the middle of the row; a unit too
-  // short to split runs whole in the pair's first CTA (both decide alike,
-  // before any cluster-wide step)
-  int kb0 = 0, kb1 = nblk;
-  bool paired = false;
-  if (p.split) {
-    int kmid = 0;
-    if (nblk > kSegBlocks) {
-      const int c = (nblk + kSegBlocks) / (2 * kSegBlocks);   // nearest segment count to the middle
-      kmid = kSegBlocks * max(1, min(c, (nblk - 1) / kSegBlocks));
-    }
-    if (kmid == 0) {
-      if (half) return;
-    } else {
-      paired = true;
-      if (half) kb0 = kmid;
-      else kb1 = kmid;
-    }
-  }
-  const int nkv = kb1 - kb0;
-  const bool last_partial = kb1 == nblk && (len & 127) != 0;   // this CTA holds the ragged V tile
-  // a paired CTA's softmax leaves its (scale, l) here for the combine
-  float fin_f = 0.0f, fin_l = 0.0f;
-  bool fin_ok = false;
+  const int nkv = (len + 127) / 128;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars.q_full, 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&bars.k_full[s], 1);
       mbar_init(&bars.v_full[s], 1);
-      mbar_init(&bars.k_empty[s], 2);   // one commit per MMA warp
-      mbar_init(&bars.v_empty[s], 2);
+      mbar_init(&bars.k_empty[s], ntiles);   // one commit per active MMA warp
+      mbar_init(&bars.v_empty[s], ntiles);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.s_full[i], 1);
@@ -615,8 +585,8 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_expect_tx(&bars.q_full, 2 * C::kTile);
-      for (int i = 0; i < 2; ++i)
+      mbar_expect_tx(&bars.q_full, ntiles * C::kTile);
+      for (int i = 0; i < ntiles; ++i)
         tma_load_3d(sq + i * C::kTile, &tm_q, &bars.q_full, 0, h, seq0 + q0 + 128 * i);
     }
     // K and V stages are released separately: a K stage as soon as the two
@@ -635,7 +605,7 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (jk < C::kStages || mbar_test_now(&bars.k_empty[st], ((jk / C::kStages) - 1) & 1)) {
           if (leader) {
             mbar_expect_tx(&bars.k_full[st], C::kTile);
-            tma_load_3d(sk + st * C::kTile, &tm_k, &bars.k_full[st], 0, h, seq0 + 128 * (kb0 + jk));
+            tma_load_3d(sk + st * C::kTile, &tm_k, &bars.k_full[st], 0, h, seq0 + 128 * jk);
           }
           ++jk;
           progressed = true;
@@ -646,7 +616,7 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (jv < C::kStages || mbar_test_now(&bars.v_empty[st], ((jv / C::kStages) - 1) & 1)) {
           if (leader) {
             mbar_expect_tx(&bars.v_full[st], C::kTile);
-            tma_load_3d(sv + st * C::kTile, &tm_v, &bars.v_full[st], 0, h, seq0 + 128 * (kb0 + jv));
+            tma_load_3d(sv + st * C::kTile, &tm_v, &bars.v_full[st], 0, h, seq0 + 128 * jv);
           }
           ++jv;
           progressed = true;
@@ -670,7 +640,7 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int j = (jv > C::kStages ? jv - C::kStages : 0); j < jv; ++j)
       mbar_wait(&bars.v_full[j % C::kStages], (j / C::kStages) & 1, nullptr);
     mbar_wait(&bars.q_full, 0, nullptr);
-  } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
+  } else if ((warp == kMmaWarp || warp == kMmaWarp + 1) && warp - kMmaWarp < ntiles) {
     // ------------------------------------------------------------ MMA issuers
     const int i = warp - kMmaWarp;   // query tile of this warp
     const bool leader = lane == 0;
@@ -734,7 +704,7 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         issue_s(j + 1);
       }
       ok = mbar_wait(&bars.v_full[st], (j / C::kStages) & 1, abort_flag);
-      if (ok && j + 1 == nkv && last_partial) {
+      if (ok && j + 1 == nkv && (len & 127)) {
         // tile 0's warp zeroes the rows past the sequence; tile 1's waits for it
         if (i == 0) {
           zero_tail_rows(sv + st * C::kTile, len & 127, lane);
@@ -753,7 +723,7 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (elect_one()) mma_commit(&bars.drain[i]);
     __syncwarp();
     mbar_wait(&bars.drain[i], 0, nullptr);
-  } else {
+  } else if (warp < 4 * ntiles) {
     // ------------------------------------------------------------ softmax
     const int wg = warp >> 2;
     const int wq = warp & 3;
@@ -765,8 +735,7 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
     uint8_t* prow0 = sp + (2 * wg) * C::kTile + (row >> 3) * 1024 + (row & 7) * 128;
     const float cscale = __ldg(p.descale + 0) * __ldg(p.descale + 1) * p.softmax_scale * kLog2e;
     const float ds_v = __ldg(p.descale + 2);
-    float r_run = -INFINITY;   // the P rule's reference (log2 units)
-    float f_run = -INFINITY;   // the scale O and l are held on (= r_run but for dropped blocks)
+    float m_run = -INFINITY;
     float l_run = 0.0f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
@@ -780,7 +749,7 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&bars.s_free[wg]);   // the MMA warp may compute S_i(j+1) now
-      const int valid = len - 128 * (kb0 + j);
+      const int valid = len - 128 * j;
       if (valid < 128) {
 #pragma unroll
         for (int c = 0; c < 128; ++c)
@@ -795,20 +764,15 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         mx3 = fmax3(mx3, __uint_as_float(u[c + 6]), __uint_as_float(u[c + 7]));
       }
       const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3));
-      // reference max: this block's max at the first block of a segment (and
-      // while it is -inf), else moved to it only when that exceeds it by more
-      // than kRefLag.  O and l follow the reference unless it lies more than
-      // kMaxDrop below their scale; then the block's P is dropped (all codes 0).
+      // reference max: moves to this block's max only when that exceeds it
+      // by more than kRefLag (always on the first block, m_run = -inf)
       const float m_blk = mx * cscale;
-      const bool seg_start = ((kb0 + j) & (kSegBlocks - 1)) == 0;
-      const float r_new = (seg_start || m_blk > r_run + kRefLag) ? m_blk : r_run;
-      const bool live = r_new >= f_run - kMaxDrop;
-      const float f_new = live ? r_new : f_run;
-      const bool moved = f_new != f_run;
+      const bool moved = m_blk > m_run + kRefLag;
+      const float m_new = moved ? m_blk : m_run;
       uint32_t pw[32];
       float sum;
       if (kRule == kPRuleExp2) {
-        const float neg = live ? kPOffsetLog2 - r_new : -INFINITY;
+        const float neg = kPOffsetLog2 - m_new;
         const uint64_t c2 = f2_pack(cscale, cscale);
         const uint64_t n2 = f2_pack(neg, neg);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
@@ -843,7 +807,7 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         // values of the codes (pairs summed exactly in f16 first where
         // representable, then in fp32).
         const float a16 = cscale * 0.0625f;
-        const float b16 = live ? 0.75f - r_new * 0.0625f : -INFINITY;
+        const float b16 = 0.75f - m_new * 0.0625f;
         const uint64_t magic2 = f2_pack(98304.0f, 98304.0f);   // 1.5 * 2^16
         float lacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         uint32_t hprev = 0;
@@ -873,9 +837,7 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
             make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
       fence_proxy_async();
-      // 0 on the first block, 1 unless the scale moved (above 1 only after a
-      // segment restart, and then at most 2^kMaxDrop)
-      const float alpha = moved ? ex2_approx(f_run - f_new) : 1.0f;
+      const float alpha = ex2_approx(m_run - m_new);   // 0 on the first block, 1 unless moved
       l_run = l_run * alpha + sum;
       if (j > 0 && __any_sync(0xFFFFFFFFu, moved)) {
         // O_i holds PV up to block j-1: wait for it before rescaling
@@ -903,8 +865,7 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         tmem_st_wait();
       }
-      r_run = r_new;
-      f_run = f_new;
+      m_run = m_new;
       tc_fence_before();
       mbar_arrive(&bars.p_full[wg][j & 1]);
     }
@@ -912,16 +873,12 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (lane == 0) note_error(p, bars, kErrTimeout);
     } else if (mbar_wait(&bars.pv_done[wg][(nkv - 1) & 1], ((nkv - 1) >> 1) & 1, abort_flag)) {
       tc_fence_after();
-      fin_ok = true;
-      fin_f = f_run;
-      fin_l = l_run;
       const int qrow = q0 + 128 * wg + row;
       const bool store = qrow < len;
       const float inv = ds_v / l_run;
       __nv_bfloat16* dst = p.out + (static_cast<int64_t>(seq0 + qrow) * p.H + h) * kHeadDim;
-      // a paired CTA keeps O in TMEM for the combine with the other half of the row
 #pragma unroll
-      for (int c = 0; c < (paired ? 0 : 4); ++c) {
+      for (int c = 0; c < 4; ++c) {
         uint32_t o[32];
         tmem_ld32(tO + 32 * c, o);
         tmem_ld_wait();
@@ -948,77 +905,6 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (paired) {
-    // Combine the two halves of each row on the larger scale F:
-    //   out = (O_a 2^(f_a - F) + O_b 2^(f_b - F)) ds_v / (l_a 2^(f_a - F) + l_b 2^(f_b - F)).
-    // CTA 0 finishes columns 0..63 and CTA 1 columns 64..127; each sends the
-    // other half of its O rows and its (f, l) into the peer's K/V stage
-    // buffers, free once both CTAs are past their main loops (first cluster
-    // barrier); the second barrier makes the writes visible.  Every thread
-    // of both CTAs takes both barriers on every path.
-    float* recv = reinterpret_cast<float*>(sk);   // [256 rows][64] (16-byte chunks swizzled), then [256][2]
-    const uint32_t peer = static_cast<uint32_t>(half ^ 1);
-    const int wg = warp >> 2;
-    const int rr = 128 * wg + 32 * (warp & 3) + lane;   // row of the unit (softmax threads)
-    const uint32_t tO = tmem + 256 + 128 * wg + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
-    cluster_sync();
-    if (warp < 8 && fin_ok) {
-      uint32_t o[64];
-      const uint32_t send_col = half ? 0u : 64u;
-      tmem_ld32(tO + send_col, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
-      tmem_ld32(tO + send_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
-      tmem_ld_wait();
-      const uint32_t dst = mapa_shared(smem_u32(recv + 64 * rr), peer);
-#pragma unroll
-      for (int c = 0; c < 16; ++c)
-        st_cluster_v4(dst + ((c ^ (rr & 7)) << 4), o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-      st_cluster_v2f(mapa_shared(smem_u32(recv + 64 * 256 + 2 * rr), peer), fin_f, fin_l);
-    }
-    cluster_sync();
-    if (warp < 8 && fin_ok) {
-      const float pf = recv[64 * 256 + 2 * rr];
-      const float pl = recv[64 * 256 + 2 * rr + 1];
-      // the same sum in both CTAs: the first CTA's term first
-      const float fa = half ? pf : fin_f, fb = half ? fin_f : pf;
-      const float la = half ? pl : fin_l, lb = half ? fin_l : pl;
-      const float F = fmaxf(fa, fb);
-      const float wa = fa == F ? 1.0f : ex2_approx(fa - F);
-      const float wb = fb == F ? 1.0f : ex2_approx(fb - F);
-      const float inv = __ldg(p.descale + 2) / (la * wa + lb * wb);
-      const float w_me = (half ? wb : wa) * inv, w_pe = (half ? wa : wb) * inv;
-      const uint32_t keep_col = half ? 64u : 0u;
-      const int qrow = q0 + rr;
-      __nv_bfloat16* dst = p.out + (static_cast<int64_t>(seq0 + qrow) * p.H + h) * kHeadDim + keep_col;
-      const uint64_t wm2 = f2_pack(w_me, w_me), wp2 = f2_pack(w_pe, w_pe);
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tO + keep_col + 32 * c, o);
-        tmem_ld_wait();
-        uint32_t w[16];
-#pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          const float4 pv = *reinterpret_cast<const float4*>(
-              recv + 64 * rr + 4 * ((8 * c + x) ^ (rr & 7)));
-          float o0, o1, o2, o3;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(o[4 * x]), __uint_as_float(o[4 * x + 1])), wm2,
-                           f2_mul(f2_pack(pv.x, pv.y), wp2)), o0, o1);
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(o[4 * x + 2]), __uint_as_float(o[4 * x + 3])), wm2,
-                           f2_mul(f2_pack(pv.z, pv.w), wp2)), o2, o3);
-          w[2 * x] = cvt_bf16x2(o0, o1);
-          w[2 * x + 1] = cvt_bf16x2(o2, o3);
-        }
-        if (qrow < len) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
-#pragma unroll
-          for (int x = 0; x < 4; ++x) d4[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
-        }
-      }
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-  }
   if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
@@ -1131,46 +1017,26 @@ bool make_qkv_map(CUtensorMap* m, const void* base, int64_t T, int H, bool bf16)
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// How many of a launch's `grid` units run as CTA pairs (the last ones).
-// Auto: the units of a last wave that is at most half full (so the pairs
-// fit in one wave beside nothing else), when every pair can be resident at
-// once; none when no sequence is longer than one segment.
-int64_t split_pairs(void (*kernel)(CUtensorMap, CUtensorMap, CUtensorMap, AttnParams),
-                    int smem_bytes, int64_t grid, int max_seqlen, int schedule, int dev) {
-  if (schedule == kSchedWhole || max_seqlen <= kSegBlocks * 128) return 0;
-  if (schedule == kSchedSplit) return grid;
+// How many of a launch's `units` (the last ones) run as two single-tile
+// CTAs each.  Auto: the units of a last wave that would fill at most half
+// of the SMs, so that their tiles fill that wave instead.
+int64_t split_units(int64_t units, int schedule, int dev) {
+  if (schedule == kSchedWhole) return 0;
+  if (schedule == kSchedSplit) return units;
   static std::mutex mu;
   static int n_sm[64] = {0};
-  static int n_clusters[64] = {0};
+  int sms;
   {
     std::lock_guard<std::mutex> lock(mu);
-    if (n_sm[dev] == 0) {
-      int sms = 0, nc = 0;
-      if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return 0;
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(2);
-      cfg.blockDim = dim3(kThreadsFp8);
-      cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = 2;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      if (cudaOccupancyMaxActiveClusters(&nc, reinterpret_cast<const void*>(kernel), &cfg) !=
-          cudaSuccess) {
-        (void)cudaGetLastError();
-        nc = 0;
-      }
-      n_clusters[dev] = nc;
-      n_sm[dev] = sms;
+    if (n_sm[dev] == 0 &&
+        cudaDeviceGetAttribute(&n_sm[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      n_sm[dev] = 0;
+      return 0;
     }
+    sms = n_sm[dev];
   }
-  const int64_t sms = n_sm[dev];
-  const int64_t tail = grid % sms;
-  if (grid <= sms || tail == 0 || 2 * tail > sms || tail > n_clusters[dev]) return 0;
+  const int64_t tail = units % sms;
+  if (units <= sms || tail == 0 || 2 * tail > sms) return 0;
   return tail;
 }
 
@@ -1210,42 +1076,15 @@ cudaError_t launch_attention_t(const AttnLaunch& a, int64_t T, cudaStream_t stre
   p.softmax_scale = a.softmax_scale;
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.err = a.err;
-  p.unit0 = 0;
-  p.split = 0;
-  const int64_t grid = static_cast<int64_t>(p.n_qblk) * a.heads * a.batch;
-  if (grid <= 0) return cudaSuccess;
-  if (grid > 0x3FFFFFFF) return cudaErrorInvalidConfiguration;
-  const int64_t pairs =
-      kFp8 ? split_pairs(kernel, smem_bytes, grid, a.max_seqlen, a.schedule, dev) : 0;
-  const int64_t whole = grid - pairs;
-  if (whole > 0) {
-    kernel<<<static_cast<unsigned>(whole), kFp8 ? kThreadsFp8 : kThreadsAttn, smem_bytes,
-             stream>>>(mq, mk, mv, p);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  if (pairs > 0) {
-    // the last `pairs` units, each on a cluster of two CTAs
-    AttnParams ps = p;
-    ps.unit0 = static_cast<int>(whole);
-    ps.split = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
-    cfg.blockDim = dim3(kThreadsFp8);
-    cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, mq, mk, mv, ps);
-    if (e != cudaSuccess) return e;
-    if (whole > 0) note_launch();   // the caller counts one launch
-  }
-  return cudaSuccess;
+  const int64_t units = static_cast<int64_t>(p.n_qblk) * a.heads * a.batch;
+  if (units <= 0) return cudaSuccess;
+  if (units > 0x3FFFFFFF) return cudaErrorInvalidConfiguration;
+  const int64_t split = kFp8 ? split_units(units, a.schedule, dev) : 0;
+  p.n_whole = static_cast<int>(units - split);
+  const int64_t grid = units + split;   // whole units first, then two CTAs per split unit
+  kernel<<<static_cast<unsigned>(grid), kFp8 ? kThreadsFp8 : kThreadsAttn, smem_bytes, stream>>>(
+      mq, mk, mv, p);
+  return cudaGetLastError();
 }
 
 }  // namespace

@@ -55,8 +55,8 @@ constexpr int kPRuleExp2 = 1;
 
 // Work schedules of the FP8 kernel (the values of fp8attn_schedule).
 constexpr int kSchedAuto = 0;    // split the units of a last wave at most half full
-constexpr int kSchedWhole = 1;   // one CTA per unit
-constexpr int kSchedSplit = 2;   // every unit long enough as a pair of CTAs
+constexpr int kSchedWhole = 1;   // one CTA per unit (256 query rows, two tiles)
+constexpr int kSchedSplit = 2;   // every unit as two single-tile CTAs
 
 cudaError_t launch_attention(const AttnLaunch& p, int64_t total_tokens, cudaStream_t stream);
 

@@ -414,53 +414,3 @@ def test_move_at_the_threshold_gives_two_results_not_an_exclusion():
     o, amb, alt, alt_amb = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0,
                                                 rows=[0], return_alternative=True)
     assert np.isnan(alt).all() and np.isfinite(amb).all()
-
-
-def test_reference_starts_afresh_at_each_4096_key_segment():
-    # Key 0 scores 2 (block 0 sets r = 2); keys 1..4095 score 0 (no move);
-    # keys 4096, 4097 score -0.125 and open block 32, the first block of the
-    # second segment, so r restarts at -0.125 there: 32 exp(s - r) = 32
-    # exactly and p~ = exp(-0.125 - 2).  Carrying r = 2 into the segment would
-    # give e4m3(32 e^-2.125)/32 = e4m3(3.82)/32 = 3.75/32 instead.
-    D, n = 128, 4098
-    q8 = np.zeros((n, 1, D), np.uint8)
-    k8 = np.zeros((n, 1, D), np.uint8)
-    v8 = np.zeros((n, 1, D), np.uint8)
-    q8[:, 0, 0] = 0x38                # 1.0
-    k8[0, 0, 0] = 0x40                # 2.0
-    k8[4096:, 0, 0] = 0xA0            # -0.125
-    v8[4096, 0, 3] = 0x38
-    cu = np.array([0, n], dtype=np.int32)
-    o = oracle.attention_fp8(q8, k8, v8, cu, (1.0, 1.0, 1.0), scale=1.0, pquant=True,
-                             rows=[0], rule=oracle.P_EXP2)
-    l = 1.0 + 4095 * math.exp(-2.0) + 2 * math.exp(-2.125)
-    assert abs(o[0, 0, 3] - math.exp(-2.125) / l) < 1e-15
-    assert abs(o[0, 0, 3] - 3.75 / 32.0 / l) > 1e-6
-
-
-@pytest.mark.parametrize("rule", [oracle.P_LINEAR_LOG, oracle.P_EXP2])
-def test_segments_are_independent_a_repeated_segment_changes_nothing(rule):
-    # A row whose 8192 keys are one 4096-key segment written twice has, with
-    # the reference restarting at key 4096, two identical halves (same codes
-    # against the same references), so its output equals that of the
-    # segment alone.  The key scale grows over the blocks, so the reference
-    # moves inside the segment and a reference carried over from the first
-    # half would quantise the second half differently.
-    D, n = 128, 4096
-    g = torch.Generator().manual_seed(11)
-    growth = (1.0 + torch.arange(n) // 128 / 4.0).view(n, 1, 1)
-    k = (torch.randn(n, 1, D, generator=g) * growth).to(torch.float8_e4m3fn).view(torch.uint8)
-    v8 = _codes((n, 1, D), 12)
-    q8 = _codes((4, 1, D), 13)
-    k8 = k.numpy()
-    rows = np.arange(4, dtype=np.int64)
-    one = oracle.attention_fp8(np.concatenate([q8, np.zeros((n - 4, 1, D), np.uint8)]), k8, v8,
-                               np.array([0, n], np.int32), (0.5, 0.5, 1.0), rows=rows, rule=rule)
-    q2 = np.concatenate([q8, np.zeros((2 * n - 4, 1, D), np.uint8)])
-    two = oracle.attention_fp8(q2, np.concatenate([k8, k8]), np.concatenate([v8, v8]),
-                               np.array([0, 2 * n], np.int32), (0.5, 0.5, 1.0), rows=rows,
-                               rule=rule)
-    assert np.max(np.abs(two - one)) < 1e-12
-    # the reference does move within the segment: the output is not the
-    # one of a segment whose blocks all share block 0's reference
-    assert np.max(np.abs(one)) > 0.0

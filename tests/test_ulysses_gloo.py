@@ -52,7 +52,9 @@ def _oracle_kernels(qar):
     import oracle
     import synthetic
 
-    def varlen_fwd(q8, k8, v8, cu, max_seqlen, descale, softmax_scale=0.0, p_rule=1):
+    def varlen_fwd(q8, k8, v8, cu, max_seqlen, descale, softmax_scale=0.0, p_rule=1,
+                   schedule=qar.SCHED_AUTO):
+        # the oracle evaluates each row whole; every schedule computes that rule
         rule = oracle.P_EXP2 if p_rule == qar.P_EXP2 else oracle.P_LINEAR_LOG
         return torch.from_numpy(oracle.attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(),
                                                      np.asarray(cu), descale, rule=rule))
