@@ -506,7 +506,9 @@ struct Fp8Barriers {
   int abort_flag;
 };
 
-template <int kRule>
+// kMixed: the grid holds single-tile CTAs after the whole units (n_whole);
+// a grid of whole units only is compiled without that case.
+template <int kRule, bool kMixed>
 __global__ void __launch_bounds__(kThreadsFp8, 1)
 attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -527,9 +529,10 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
   // work unit = (query block of 256 rows, head, sequence); a CTA past
   // n_whole takes one 128-row half of a unit (ntiles = 1)
   const int cta = static_cast<int>(blockIdx.x);
-  const int ntiles = cta < p.n_whole ? 2 : 1;
-  const int unit = cta < p.n_whole ? cta : p.n_whole + ((cta - p.n_whole) >> 1);
-  const int sub = cta < p.n_whole ? 0 : ((cta - p.n_whole) & 1);
+  const bool whole = !kMixed || cta < p.n_whole;
+  const int ntiles = whole ? 2 : 1;
+  const int unit = whole ? cta : p.n_whole + ((cta - p.n_whole) >> 1);
+  const int sub = whole ? 0 : ((cta - p.n_whole) & 1);
   const int qb = unit % p.n_qblk;
   const int bh = unit / p.n_qblk;
   const int h = bh % p.H;
@@ -1040,14 +1043,15 @@ int64_t split_units(int64_t units, int schedule, int dev) {
   return tail;
 }
 
-template <bool kFp8, int kRule>
-cudaError_t launch_attention_t(const AttnLaunch& a, int64_t T, cudaStream_t stream) {
+template <bool kFp8, int kRule, bool kMixed>
+cudaError_t launch_attention_t(const AttnLaunch& a, int64_t T, cudaStream_t stream,
+                               int64_t split) {
   CUtensorMap mq, mk, mv;
   if (!make_qkv_map(&mq, a.q, T, a.heads, !kFp8) || !make_qkv_map(&mk, a.k, T, a.heads, !kFp8) ||
       !make_qkv_map(&mv, a.v, T, a.heads, !kFp8))
     return cudaErrorInvalidValue;
   // FP8 runs the P-in-shared-memory kernel; BF16 keeps P in TMEM
-  auto kernel = kFp8 ? attn_fwd_fp8_kernel<kRule> : attn_fwd_bf16_kernel;
+  auto kernel = kFp8 ? attn_fwd_fp8_kernel<kRule, kMixed> : attn_fwd_bf16_kernel;
   const int smem_bytes = kFp8 ? Fp8Cfg::kSmemBytes : Bf16Cfg::kSmemBytes;
   // the shared-memory opt-in is a per-device function attribute: set it once
   // for each device this process launches on
@@ -1077,9 +1081,6 @@ cudaError_t launch_attention_t(const AttnLaunch& a, int64_t T, cudaStream_t stre
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.err = a.err;
   const int64_t units = static_cast<int64_t>(p.n_qblk) * a.heads * a.batch;
-  if (units <= 0) return cudaSuccess;
-  if (units > 0x3FFFFFFF) return cudaErrorInvalidConfiguration;
-  const int64_t split = kFp8 ? split_units(units, a.schedule, dev) : 0;
   p.n_whole = static_cast<int>(units - split);
   const int64_t grid = units + split;   // whole units first, then two CTAs per split unit
   kernel<<<static_cast<unsigned>(grid), kFp8 ? kThreadsFp8 : kThreadsAttn, smem_bytes, stream>>>(
@@ -1104,9 +1105,21 @@ cudaError_t launch_qk_scores_probe(const void* q8, const void* k8, int64_t tiles
 }
 
 cudaError_t launch_attention(const AttnLaunch& a, int64_t total_tokens, cudaStream_t stream) {
-  if (a.bf16) return launch_attention_t<false, kPRuleExp2>(a, total_tokens, stream);
-  if (a.p_rule == kPRuleExp2) return launch_attention_t<true, kPRuleExp2>(a, total_tokens, stream);
-  return launch_attention_t<true, kPRuleLinearLog>(a, total_tokens, stream);
+  const int64_t units = static_cast<int64_t>((a.max_seqlen + 255) / 256) * a.heads * a.batch;
+  if (units <= 0) return cudaSuccess;
+  if (units > 0x3FFFFFFF) return cudaErrorInvalidConfiguration;
+  if (a.bf16) return launch_attention_t<false, kPRuleExp2, false>(a, total_tokens, stream, 0);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  const int64_t split = split_units(units, a.schedule, dev);
+  if (a.p_rule == kPRuleExp2)
+    return split ? launch_attention_t<true, kPRuleExp2, true>(a, total_tokens, stream, split)
+                 : launch_attention_t<true, kPRuleExp2, false>(a, total_tokens, stream, 0);
+  return split ? launch_attention_t<true, kPRuleLinearLog, true>(a, total_tokens, stream, split)
+               : launch_attention_t<true, kPRuleLinearLog, false>(a, total_tokens, stream, 0);
 }
+
 
 }  // namespace fp8attn
