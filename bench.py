@@ -826,6 +826,17 @@ def run_ours(args):
                        p_rule=P_RULES[args.p_rule], schedule=qar.SCHED_WHOLE)
     attn_whole()
     whole_s = _time_launches(attn_whole, dev, stream, 20, flush_l2)
+
+    # the library's bf16 attention (the skip-layer kernel) on the same bf16
+    # inputs: the FP8 path's speed-up over native-dtype attention
+    out_bf = torch.empty_like(out)
+
+    def attn_bf16():
+        qar.varlen_fwd_bf16(q, k, v, cu_d, S, out=out_bf, stream=stream)
+    attn_bf16()
+    bf16_s = _time_launches(attn_bf16, dev, stream, 20, flush_l2)
+    fp8_alone_s = _time_launches(attn, dev, stream, 20, flush_l2)   # timed the same way
+    del out_bf
     per_config = None
     if world == 1 and not args.no_per_config:
         per_config = measure_per_config(dev, stream, p_rule, fp8_peak, flush_l2)
@@ -857,6 +868,10 @@ def run_ours(args):
                                 "attn_tflops": FLOPS_PER_STEP / other_s / 1e12},
             "attn_whole_units": {"schedule": "one CTA per unit", "attn_us": whole_s * 1e6,
                                  "attn_tflops": FLOPS_PER_STEP / whole_s / 1e12},
+            "attn_bf16": {"kernel": "attn_fwd_bf16_kernel (bf16 Q/K/V, no quantisation)",
+                          "attn_us": bf16_s * 1e6, "attn_tflops": FLOPS_PER_STEP / bf16_s / 1e12,
+                          "fp8_attn_us_timed_alike": fp8_alone_s * 1e6,
+                          "fp8_speedup": bf16_s / fp8_alone_s},
             "err_vs_unquantized": err_uq,
             "quant_us": quant_s * 1e6, "quant_gbs": quant_gbs,
             "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": fp8_peak,
