@@ -242,7 +242,8 @@ typedef enum {
  *   FP8ATTN_SCHED_AUTO: one CTA per unit, except that when the last wave of
  *     units would fill at most half of the SMs, each of those units runs as
  *     two CTAs of one tile each, so that the tiles fill that wave (a lone
- *     tile's blocks run faster than a CTA's two interleaved tiles).
+ *     tile's blocks run faster than a CTA's two interleaved tiles); those
+ *     CTAs form a second launch that starts as SMs free up.
  *   FP8ATTN_SCHED_WHOLE: one CTA per unit.
  *   FP8ATTN_SCHED_SPLIT: every unit as two single-tile CTAs. */
 typedef enum {

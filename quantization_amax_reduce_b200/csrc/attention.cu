@@ -72,10 +72,7 @@ struct Bf16Cfg {
 struct AttnParams {
   const int32_t* cu;
   int B, H, max_seqlen, n_qblk;   // n_qblk = query blocks of 256 rows per sequence
-  // FP8: CTAs [0, n_whole) each run one work unit (256 query rows of one
-  // head) as two 128-row tiles; every CTA after them runs one tile of the
-  // units from n_whole on (two CTAs per unit)
-  int n_whole;
+  int unit0;   // FP8: the launch's first work unit (256 query rows of one head)
   int64_t T;
   const float* descale;
   float softmax_scale;
@@ -506,9 +503,10 @@ struct Fp8Barriers {
   int abort_flag;
 };
 
-// kMixed: the grid holds single-tile CTAs after the whole units (n_whole);
-// a grid of whole units only is compiled without that case.
-template <int kRule, bool kMixed>
+// kSplit = 0: each CTA runs one work unit as two interleaved 128-row tiles.
+// kSplit = 1: each unit runs as two CTAs of one tile each.  The two are
+// separate instantiations so that each compiles with its tile count fixed.
+template <int kRule, int kSplit>
 __global__ void __launch_bounds__(kThreadsFp8, 1)
 attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -526,13 +524,14 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // work unit = (query block of 256 rows, head, sequence); a CTA past
-  // n_whole takes one 128-row half of a unit (ntiles = 1)
+  // a launch of single-tile CTAs may follow this grid on the stream: let it
+  // start as soon as SMs free up (it reads nothing this grid writes)
+  if (kSplit == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // work unit = (query block of 256 rows, head, sequence)
   const int cta = static_cast<int>(blockIdx.x);
-  const bool whole = !kMixed || cta < p.n_whole;
-  const int ntiles = whole ? 2 : 1;
-  const int unit = whole ? cta : p.n_whole + ((cta - p.n_whole) >> 1);
-  const int sub = whole ? 0 : ((cta - p.n_whole) & 1);
+  constexpr int ntiles = kSplit ? 1 : 2;
+  const int unit = p.unit0 + (kSplit ? (cta >> 1) : cta);
+  const int sub = kSplit ? (cta & 1) : 0;
   const int qb = unit % p.n_qblk;
   const int bh = unit / p.n_qblk;
   const int h = bh % p.H;
@@ -543,10 +542,14 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
   if (seq0 < 0 || len < 0 || len > p.max_seqlen || static_cast<int64_t>(seq1) > p.T) {
     if (threadIdx.x == 0 && qb == 0 && sub == 0 && p.err)
       atomicOr(reinterpret_cast<unsigned int*>(p.err), kErrSeqlens);
+    if (kSplit) asm volatile("griddepcontrol.wait;" ::: "memory");
     return;
   }
   const int q0 = qb * 256 + 128 * sub;   // first query row of this CTA's tile 0
-  if (q0 >= len) return;
+  if (q0 >= len) {
+    if (kSplit) asm volatile("griddepcontrol.wait;" ::: "memory");
+    return;
+  }
   const int nkv = (len + 127) / 128;
 
   if (threadIdx.x == 0) {
@@ -909,6 +912,9 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
   __syncthreads();
   tc_fence_after();
   if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+  // a single-tile grid launched behind a grid of whole units finishes only
+  // after that grid (later work on the stream then follows both)
+  if (kSplit) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -1043,15 +1049,17 @@ int64_t split_units(int64_t units, int schedule, int dev) {
   return tail;
 }
 
-template <bool kFp8, int kRule, bool kMixed>
+// Launches `n_units` work units from `unit0` on (kSplit: two single-tile CTAs
+// per unit; `behind`: programmatic launch behind the previous kernel).
+template <bool kFp8, int kRule, int kSplit>
 cudaError_t launch_attention_t(const AttnLaunch& a, int64_t T, cudaStream_t stream,
-                               int64_t split) {
+                               int64_t unit0, int64_t n_units, bool behind) {
   CUtensorMap mq, mk, mv;
   if (!make_qkv_map(&mq, a.q, T, a.heads, !kFp8) || !make_qkv_map(&mk, a.k, T, a.heads, !kFp8) ||
       !make_qkv_map(&mv, a.v, T, a.heads, !kFp8))
     return cudaErrorInvalidValue;
   // FP8 runs the P-in-shared-memory kernel; BF16 keeps P in TMEM
-  auto kernel = kFp8 ? attn_fwd_fp8_kernel<kRule, kMixed> : attn_fwd_bf16_kernel;
+  auto kernel = kFp8 ? attn_fwd_fp8_kernel<kRule, kSplit> : attn_fwd_bf16_kernel;
   const int smem_bytes = kFp8 ? Fp8Cfg::kSmemBytes : Bf16Cfg::kSmemBytes;
   // the shared-memory opt-in is a per-device function attribute: set it once
   // for each device this process launches on
@@ -1080,12 +1088,24 @@ cudaError_t launch_attention_t(const AttnLaunch& a, int64_t T, cudaStream_t stre
   p.softmax_scale = a.softmax_scale;
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.err = a.err;
-  const int64_t units = static_cast<int64_t>(p.n_qblk) * a.heads * a.batch;
-  p.n_whole = static_cast<int>(units - split);
-  const int64_t grid = units + split;   // whole units first, then two CTAs per split unit
-  kernel<<<static_cast<unsigned>(grid), kFp8 ? kThreadsFp8 : kThreadsAttn, smem_bytes, stream>>>(
-      mq, mk, mv, p);
-  return cudaGetLastError();
+  p.unit0 = static_cast<int>(unit0);
+  const int64_t grid = kSplit ? 2 * n_units : n_units;
+  const int threads = kFp8 ? kThreadsFp8 : kThreadsAttn;
+  if (!behind) {
+    kernel<<<static_cast<unsigned>(grid), threads, smem_bytes, stream>>>(mq, mk, mv, p);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, mq, mk, mv, p);
 }
 
 }  // namespace
@@ -1104,21 +1124,31 @@ cudaError_t launch_qk_scores_probe(const void* q8, const void* k8, int64_t tiles
   return cudaGetLastError();
 }
 
+template <int kRule>
+cudaError_t launch_fp8(const AttnLaunch& a, int64_t T, cudaStream_t stream, int64_t units,
+                       int64_t split) {
+  // whole units first, then the split units' single-tile CTAs behind them
+  const int64_t whole = units - split;
+  if (whole > 0) {
+    cudaError_t e = launch_attention_t<true, kRule, 0>(a, T, stream, 0, whole, false);
+    if (e != cudaSuccess || split == 0) return e;
+    note_launch();   // the caller counts one launch
+  }
+  return launch_attention_t<true, kRule, 1>(a, T, stream, whole, split, whole > 0);
+}
+
 cudaError_t launch_attention(const AttnLaunch& a, int64_t total_tokens, cudaStream_t stream) {
   const int64_t units = static_cast<int64_t>((a.max_seqlen + 255) / 256) * a.heads * a.batch;
   if (units <= 0) return cudaSuccess;
   if (units > 0x3FFFFFFF) return cudaErrorInvalidConfiguration;
-  if (a.bf16) return launch_attention_t<false, kPRuleExp2, false>(a, total_tokens, stream, 0);
+  if (a.bf16) return launch_attention_t<false, kPRuleExp2, 0>(a, total_tokens, stream, 0, units, false);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   const int64_t split = split_units(units, a.schedule, dev);
-  if (a.p_rule == kPRuleExp2)
-    return split ? launch_attention_t<true, kPRuleExp2, true>(a, total_tokens, stream, split)
-                 : launch_attention_t<true, kPRuleExp2, false>(a, total_tokens, stream, 0);
-  return split ? launch_attention_t<true, kPRuleLinearLog, true>(a, total_tokens, stream, split)
-               : launch_attention_t<true, kPRuleLinearLog, false>(a, total_tokens, stream, 0);
+  return a.p_rule == kPRuleExp2 ? launch_fp8<kPRuleExp2>(a, total_tokens, stream, units, split)
+                                : launch_fp8<kPRuleLinearLog>(a, total_tokens, stream, units, split);
 }
 
 
