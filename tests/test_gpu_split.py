@@ -94,3 +94,49 @@ def test_scores_spanning_hundreds_of_log2_units(rule, orule, start):
     assert torch.isfinite(outs["whole"].float()).all()
     assert_attention_close(outs["whole"], want, rows=rows,
                            what=f"score range from {start}, {orule}")
+
+
+def _split_sized_case(seed):
+    # 512 units (S=8192, 16 heads): on 148 SMs the automatic schedule runs
+    # the last 68 as single-tile CTAs in a second launch behind the first
+    S, H = 8192, 16
+    q8, k8, v8 = (_codes(S, H, seed + s, 6.0) for s in range(3))
+    return [x.to(DEV) for x in (q8, k8, v8)], torch.tensor([0, S], dtype=torch.int32, device=DEV)
+
+
+def test_split_call_in_a_cuda_graph_matches_eager():
+    (q8, k8, v8), cu = _split_sized_case(90)
+    ds = torch.tensor([0.05, 0.04, 1.0 / 60.0], device=DEV)
+    eager = qar.varlen_fwd(q8, k8, v8, cu, 8192, ds)
+    out = torch.empty_like(eager)
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        qar.varlen_fwd(q8, k8, v8, cu, 8192, ds, out=out, stream=stream)   # warm-up
+    torch.cuda.current_stream().wait_stream(stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    out.zero_()
+    with torch.cuda.graph(g, stream=stream):
+        qar.varlen_fwd(q8, k8, v8, cu, 8192, ds, out=out, stream=stream)
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, eager)
+
+
+def test_back_to_back_split_calls_keep_stream_order():
+    # two calls into the same output on one stream: every row must hold the
+    # second call's result (the first call's single-tile launch may not end
+    # after the second call has written)
+    (qa, ka, va), cu = _split_sized_case(91)
+    (qb, kb, vb), _ = _split_sized_case(95)
+    ds = torch.tensor([0.05, 0.04, 1.0 / 60.0], device=DEV)
+    want = qar.varlen_fwd(qb, kb, vb, cu, 8192, ds)
+    out = torch.empty_like(want)
+    for _ in range(3):
+        qar.varlen_fwd(qa, ka, va, cu, 8192, ds, out=out)
+        qar.varlen_fwd(qb, kb, vb, cu, 8192, ds, out=out)
+        torch.cuda.synchronize()
+        assert torch.equal(out, want)
