@@ -134,6 +134,25 @@ fp8attn_status fp8attn_quantize_qkv(fp8attn_ctx* ctx, int layer, int mode, const
                                     int64_t total_tokens, int num_heads, int head_dim, void* q8,
                                     void* k8, void* v8, void* stream);
 
+/* The cast of fp8attn_quantize_qkv (modes STATIC and RING only) writing each
+ * output head-grouped: q8, k8, v8 are [groups][total_tokens][num_heads /
+ * groups][head_dim], group g holding heads [g H/groups, (g+1) H/groups) of
+ * every token, i.e. the send buffer of the all-to-all that hands group g to
+ * rank g in sequence-parallel (Ulysses) attention (vLLM-Omni "Quantized KV
+ * Cache", Configuration: the DiT sharded over a Ulysses degree).  One launch
+ * for all groups; the codes equal those of fp8attn_quantize_qkv, regrouped.
+ * groups must divide num_heads (groups = 1 is the packed layout).  Sources,
+ * scales and errors as fp8attn_quantize_qkv; INVALID for mode DYNAMIC or
+ * SKIP (a sharded dynamic pass reduces its amax across ranks first, then
+ * casts with RING) and for a bad group count. */
+fp8attn_status fp8attn_quantize_qkv_grouped(fp8attn_ctx* ctx, int layer, int mode, const void* q,
+                                            const void* k, const void* v, int64_t tok_stride,
+                                            int64_t head_stride, const int32_t* d_src_seq_start,
+                                            const int32_t* d_cu_seqlens, int batch,
+                                            int max_seqlen, int64_t total_tokens, int num_heads,
+                                            int head_dim, int groups, void* q8, void* k8,
+                                            void* v8, void* stream);
+
 /* Per-tensor amax of Q, K and V over their valid tokens into d_amax3 (device
  * float[3]; NaN ignored, an infinite amax stays infinite), without casting
  * and without touching any ring (vLLM FP8 ViT page, usage section: the ring

@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
         "fp8attn_destroy": (I, [P]),
         "fp8attn_quantize_qkv": (I, [P, I, I, P, P, P, I64, I64, P, P, I, I, I64, I, I, P, P, P,
                                      P]),
+        "fp8attn_quantize_qkv_grouped": (I, [P, I, I, P, P, P, I64, I64, P, P, I, I, I64, I, I, I,
+                                             P, P, P, P]),
         "fp8attn_amax_ring_update": (I, [P, I, P, P]),
         "fp8attn_amax_qkv": (I, [P, P, P, P, I64, I64, P, P, I, I, I64, I, I, P, P]),
         "fp8attn_set_static_scales": (I, [P, I, F, F, F, P]),
@@ -274,6 +276,35 @@ class Context:
             _ptr(cu), B, int(max_seqlen), int(total_tokens), H, HEAD_DIM, _ptr(out[0]),
             _ptr(out[1]), _ptr(out[2]), ctypes.c_void_p(_stream(stream, q.device))),
             "fp8attn_quantize_qkv")
+        return out[0], out[1], out[2]
+
+    def quantize_qkv_grouped(self, layer: int, mode: int, q: torch.Tensor, k: torch.Tensor,
+                             v: torch.Tensor, cu_seqlens, max_seqlen: int, groups: int, *,
+                             total_tokens: Optional[int] = None, src_seq_start=None,
+                             out=None, stream=None
+                             ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+        """The STATIC or RING cast of ``quantize_qkv`` written head-grouped:
+        returns uint8 E4M3 codes [groups, T, H / groups, 128] per tensor, group
+        g holding heads [g H/groups, (g+1) H/groups) -- the send buffers of a
+        sequence-parallel all-to-all, in one launch."""
+        H, tok_stride, head_stride, cu, B, total_tokens, sss = _qkv_source(
+            q, k, v, cu_seqlens, total_tokens, src_seq_start)
+        groups = int(groups)
+        if groups < 1 or H % groups:
+            raise ValueError(f"groups {groups} must divide the {H} heads")
+        if out is None:
+            out = [torch.empty((groups, total_tokens, H // groups, HEAD_DIM), dtype=torch.uint8,
+                               device=q.device) for _ in range(3)]
+        else:
+            if len(out) != 3:
+                raise ValueError("out must hold three tensors (q8, k8, v8)")
+            for name, t in zip(("q8", "k8", "v8"), out):
+                _check_out(t, name, torch.uint8, int(total_tokens) * H * HEAD_DIM, q.device)
+        _check(lib().fp8attn_quantize_qkv_grouped(
+            self._h, layer, mode, _ptr(q), _ptr(k), _ptr(v), tok_stride, head_stride, _ptr(sss),
+            _ptr(cu), B, int(max_seqlen), int(total_tokens), H, HEAD_DIM, groups, _ptr(out[0]),
+            _ptr(out[1]), _ptr(out[2]), ctypes.c_void_p(_stream(stream, q.device))),
+            "fp8attn_quantize_qkv_grouped")
         return out[0], out[1], out[2]
 
     def amax_qkv(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens,
@@ -777,12 +808,8 @@ def ulysses_attention(ctx: "Context", layer: int, mode: int, q: torch.Tensor, k:
                 comm.all_reduce_max(amax)
                 ctx.amax_ring_update(layer, amax)
                 cast = RING
-            send = [torch.empty((n, S_loc, Hn, D), dtype=torch.uint8, device=dev)
-                    for _ in range(3)]
-            for g in range(n):
-                h = slice(g * Hn, (g + 1) * Hn)
-                ctx.quantize_qkv(layer, cast, q[:, h], k[:, h], v[:, h], cu_loc, S_loc,
-                                 out=(send[0][g], send[1][g], send[2][g]))
+            # one launch casts every head group straight into its send chunk
+            send = list(ctx.quantize_qkv_grouped(layer, cast, q, k, v, cu_loc, S_loc, n))
         if n > 1:
             recv = [torch.empty_like(x) for x in send]
             for r, x in zip(recv, send):

@@ -217,6 +217,53 @@ fp8attn_status fp8attn_quantize_qkv(fp8attn_ctx* ctx, int layer, int mode, const
   return FP8ATTN_OK;
 }
 
+fp8attn_status fp8attn_quantize_qkv_grouped(fp8attn_ctx* ctx, int layer, int mode, const void* q,
+                                            const void* k, const void* v, int64_t tok_stride,
+                                            int64_t head_stride, const int32_t* d_src_seq_start,
+                                            const int32_t* d_cu_seqlens, int batch,
+                                            int max_seqlen, int64_t total_tokens, int num_heads,
+                                            int head_dim, int groups, void* q8, void* k8,
+                                            void* v8, void* stream) {
+  if (mode != FP8ATTN_STATIC && mode != FP8ATTN_RING) return FP8ATTN_ERR_INVALID;
+  if (groups < 1 || num_heads < 1 || num_heads % groups) return FP8ATTN_ERR_INVALID;
+  if (!layer_ok(ctx, layer)) return FP8ATTN_ERR_INVALID;
+  if (mode == FP8ATTN_STATIC && !ctx->has_static[layer]) return FP8ATTN_ERR_INVALID;
+  if (batch < 1 || max_seqlen < 0 || total_tokens < 0 || !d_cu_seqlens)
+    return FP8ATTN_ERR_INVALID;
+  if (head_dim != kHeadDim) return FP8ATTN_ERR_UNSUPPORTED;
+  if (total_tokens > static_cast<int64_t>(batch) * max_seqlen) return FP8ATTN_ERR_INVALID;
+  if (!q || !k || !v || !q8 || !k8 || !v8) return FP8ATTN_ERR_INVALID;
+  if (tok_stride <= 0 || head_stride <= 0 || (tok_stride % 8) || (head_stride % 8))
+    return FP8ATTN_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(q8, 16) ||
+      !aligned(k8, 16) || !aligned(v8, 16))
+    return FP8ATTN_ERR_UNSUPPORTED;
+  QuantLaunch L;
+  L.src[0] = q;
+  L.src[1] = k;
+  L.src[2] = v;
+  L.dst[0] = q8;
+  L.dst[1] = k8;
+  L.dst[2] = v8;
+  L.tok_stride = tok_stride;
+  L.head_stride = head_stride;
+  L.cu = d_cu_seqlens;
+  L.src_seq_start = d_src_seq_start;
+  L.batch = batch;
+  L.heads = num_heads;
+  L.max_seqlen = max_seqlen;
+  L.total_tokens = total_tokens;
+  L.kind = mode == FP8ATTN_RING ? kQuantRing : kQuantStatic;
+  L.amax_out = nullptr;
+  L.gs = ctx->gs;
+  L.ls = ctx->ls + layer;
+  L.dst_groups = groups;
+  const cudaError_t e = launch_quantize(L, as_stream(stream));
+  if (e != cudaSuccess) return FP8ATTN_ERR_CUDA;
+  g_launches.fetch_add(1);
+  return FP8ATTN_OK;
+}
+
 fp8attn_status fp8attn_amax_qkv(fp8attn_ctx* ctx, const void* q, const void* k, const void* v,
                                 int64_t tok_stride, int64_t head_stride,
                                 const int32_t* d_src_seq_start, const int32_t* d_cu_seqlens,

@@ -19,6 +19,7 @@ struct QuantLaunch {
   float* amax_out;               // kQuantAmaxOnly: device float[3]
   void* gs;                      // GlobalState*
   void* ls;                      // LayerState*
+  int dst_groups = 1;            // static / ring cast: > 1 writes [groups][T][H/groups][128]
 };
 
 enum QuantKind {

@@ -38,6 +38,7 @@ struct QuantArgs {
   LayerState* ls;
   int cast_with_ring;     // static kernel: 1 = use the ring scales qs (kQuantRing)
   float* amax_out;        // amax kernel: device float[3]
+  int dst_groups;         // static kernel, kGrouped: head groups of the output
 };
 
 constexpr int kThreads = 512;
@@ -263,7 +264,20 @@ __global__ void __launch_bounds__(kThreads) quant_dynamic_kernel(QuantArgs a) {
 // stride loop with six loads in flight per step and no per-tensor tail.
 constexpr int kUnrollStatic = 2;
 
-template <bool kContig>
+// Index of output vector p (16 codes: vector p % 8 of token p / (8 H), head
+// (p / 8) % H) in the head-grouped layout [groups][T][H / groups][128]: the
+// send buffer of a sequence-parallel all-to-all, group g going to rank g.
+__device__ __forceinline__ int64_t grouped_vec(const QuantArgs& a, int64_t T, int64_t p) {
+  const int64_t per_tok = static_cast<int64_t>(a.H) * 8;
+  const int64_t tok = p / per_tok;
+  const int rem = static_cast<int>(p - tok * per_tok);
+  const int head = rem >> 3;
+  const int hn = a.H / a.dst_groups;
+  const int g = head / hn;
+  return (static_cast<int64_t>(g) * T + tok) * (hn * 8) + (head - g * hn) * 8 + (rem & 7);
+}
+
+template <bool kContig, bool kGrouped>
 __global__ void __launch_bounds__(kThreads) quant_static_kernel(QuantArgs a) {
   if (!seqlens_ok(a)) {
     if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(&a.gs->error, kErrSeqlens);
@@ -292,11 +306,12 @@ __global__ void __launch_bounds__(kThreads) quant_static_kernel(QuantArgs a) {
     for (int u = 0; u < kUnrollStatic; ++u) {
       const int64_t p = p0 + u * stride;
       if (p < npair) {
+        const int64_t d = kGrouped ? grouped_vec(a, T, p) : p;
 #pragma unroll
         for (int t = 0; t < 3; ++t) {
           const uint2 lo = cast8(x[u][t][0], qs[t]);
           const uint2 hi = cast8(x[u][t][1], qs[t]);
-          reinterpret_cast<uint4*>(a.dst[t])[p] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+          reinterpret_cast<uint4*>(a.dst[t])[d] = make_uint4(lo.x, lo.y, hi.x, hi.y);
         }
       }
     }
@@ -409,6 +424,7 @@ cudaError_t launch_quantize(const QuantLaunch& q, cudaStream_t stream) {
   a.ls = static_cast<LayerState*>(q.ls);
   a.cast_with_ring = q.kind == kQuantRing;
   a.amax_out = q.amax_out;
+  a.dst_groups = q.dst_groups;
   const bool contig = q.src_seq_start == nullptr && q.head_stride == kHeadDim &&
                       q.tok_stride == static_cast<int64_t>(q.heads) * kHeadDim;
   // enough CTAs to cover the upper bound of the work, at most one full wave
@@ -447,10 +463,16 @@ cudaError_t launch_quantize(const QuantLaunch& q, cudaStream_t stream) {
     cfg.numAttrs = 1;
     return cudaLaunchKernelExC(&cfg, fn, args);
   }
-  const void* fn = contig ? reinterpret_cast<const void*>(&quant_static_kernel<true>)
-                          : reinterpret_cast<const void*>(&quant_static_kernel<false>);
-  const int cap = contig ? max_coresident(quant_static_kernel<true>, kThreads)
-                         : max_coresident(quant_static_kernel<false>, kThreads);
+  const bool grouped = q.dst_groups > 1;
+  const void* fn =
+      grouped ? (contig ? reinterpret_cast<const void*>(&quant_static_kernel<true, true>)
+                        : reinterpret_cast<const void*>(&quant_static_kernel<false, true>))
+              : (contig ? reinterpret_cast<const void*>(&quant_static_kernel<true, false>)
+                        : reinterpret_cast<const void*>(&quant_static_kernel<false, false>));
+  const int cap = grouped ? (contig ? max_coresident(quant_static_kernel<true, true>, kThreads)
+                                    : max_coresident(quant_static_kernel<false, true>, kThreads))
+                          : (contig ? max_coresident(quant_static_kernel<true, false>, kThreads)
+                                    : max_coresident(quant_static_kernel<false, false>, kThreads));
   if (cap <= 0) return cudaErrorInvalidConfiguration;
   const int grid = static_cast<int>(want < cap ? (want < 1 ? 1 : want) : cap);
   cfg.gridDim = dim3(grid);

@@ -59,5 +59,19 @@ class OracleContext:
             res.append(codes)
         return tuple(res)
 
+    def quantize_qkv_grouped(self, layer, mode, q, k, v, cu_seqlens, max_seqlen, groups, *,
+                             total_tokens=None, src_seq_start=None, out=None, stream=None):
+        codes = self.quantize_qkv(layer, mode, q, k, v, cu_seqlens, max_seqlen,
+                                  total_tokens=total_tokens, src_seq_start=src_seq_start)
+        res = []
+        for t, c in enumerate(codes):
+            T, Hh, Dd = c.shape
+            g = c.view(T, groups, Hh // groups, Dd).permute(1, 0, 2, 3).contiguous()
+            if out is not None:
+                out[t].copy_(g)
+                g = out[t]
+            res.append(g)
+        return tuple(res)
+
     def descale_ptr(self, layer):
         return [float(d) for d in self.ds]

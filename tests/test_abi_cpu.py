@@ -116,6 +116,14 @@ def test_host_argument_checks_need_no_gpu(L):
     assert L.fp8attn_selftest_bounded_waits(ctypes.c_uint64(0), ctypes.byref(n), None) == 1
     assert L.fp8attn_selftest_bounded_waits(ctypes.c_uint64(2 * 10**9), ctypes.byref(n), None) == 1
     assert L.fp8attn_selftest_bounded_waits(ctypes.c_uint64(10**6), None, None) == 1
+    # the grouped cast: STATIC / RING only, groups dividing the heads, checked
+    # before any CUDA call (mode DYNAMIC = 0, STATIC = 1, RING = 3)
+    g = (P(16), P(16), P(16), 1024, 128, None, P(16), 1, 8, 8, 8, 128)
+    outs = (P(16), P(16), P(16), None)
+    assert L.fp8attn_quantize_qkv_grouped(P(64), 0, 0, *g, 2, *outs) == 1    # DYNAMIC
+    assert L.fp8attn_quantize_qkv_grouped(P(64), 0, 2, *g, 2, *outs) == 1    # SKIP
+    assert L.fp8attn_quantize_qkv_grouped(P(64), 0, 3, *g, 3, *outs) == 1    # 8 % 3
+    assert L.fp8attn_quantize_qkv_grouped(P(64), 0, 3, *g, 0, *outs) == 1
     # head regrouping: sizes, groups, direction, alignment and overlap are
     # checked on the host; zero tokens is a no-op
     src, dst = P(1 << 20), P(1 << 24)
