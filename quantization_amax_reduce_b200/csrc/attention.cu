@@ -6,30 +6,33 @@
 // kernel on native bf16 inputs for skipped layers (vLLM-Omni parameters
 // table: selected layers keep the native dtype).
 //
-// One CTA owns two 128-row query tiles of one (sequence, head) and streams
-// that sequence's 128-key K/V tiles once for both:
-//   warp 8       TMA producer: Q tiles once, then a ring of K/V stages
-//   warp 9       MMA issuer (one lane): S_i = Q_i K^T into TMEM, then
-//                O_i += P_i V (V in shared memory, MN-major)
-//   warps 0-3    softmax for query tile 0, warps 4-7 for tile 1: one thread
-//                per query row (= TMEM lane), row max, exp2 with the
-//                descales folded into one FMA, row sum of the unquantised
-//                p, P quantised for the PV product, O rescaled in TMEM when
-//                the max that P is taken against changes, and the bf16
-//                epilogue.
+// A work unit is 256 query rows (two 128-row tiles) of one (sequence, head);
+// its CTA streams the sequence's 128-key K/V tiles once for both tiles:
+//   warp 8        TMA producer: Q tiles once, then rings of K and V stages
+//   warps 9, 10   FP8: MMA issuers for tiles 0 and 1 (one lane each):
+//                 S_i = Q_i K^T into TMEM, then O_i += P_i V (V in shared
+//                 memory, MN-major); bf16: warp 9 issues for both tiles
+//   warps 0-3     softmax for tile 0, warps 4-7 for tile 1: one thread per
+//                 query row (= TMEM lane): block max, P quantised for the
+//                 PV product, row sum, O rescaled in TMEM when the max that
+//                 P is taken against moves, and the bf16 epilogue.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512).
 // attn_fwd_bf16_kernel: P_i aliases the first 64 columns of S_i and PV
 // reads it from TMEM; S_i(j+1) is issued after PV_i(j).
-// attn_fwd_fp8_kernel (FP8): P_i goes to shared memory, so S_i(j+1) is
-// computed while the softmax still works on block j (details there).
+// attn_fwd_fp8_kernel: P_i goes to shared memory, so S_i(j+1) is computed
+// while the softmax still works on block j.  Its <rule, 1> instantiation
+// runs a unit as two CTAs of one tile each (the automatic schedule's fill
+// for a mostly empty last wave, launched behind the whole units).
 //
 // P rule (pages silent; fixed here), per 128-key block: c = ds_q ds_k
-// softmax_scale log2(e), t = s*c; FP8: p' = 2^(t - r + 5) against a reference
-// max r that starts at the first block's max and moves to a later block's
-// max only when that exceeds r by more than 3 (so p' <= 2^8 = 256, never
-// saturating, and O is rescaled only on such moves); BF16: p' = 2^(t - m)
-// with m the running max.  P = e4m3(p') (bf16(p')) for the PV product; l
-// accumulates the unquantised p'; out = O ds_v / l.
+// softmax_scale log2(e), t = s c - r + 5 against a reference max r that
+// starts at the first block's max of s c and moves to a later block's max
+// only when that exceeds r by more than 3 (so t <= 8: P never saturates, and
+// O is rescaled only on such moves).  FP8 linear-log rule (default): the
+// E4M3 code is RNE(8 t + 56) clamped to [0, 128] and l sums the codes'
+// values; FP8 exp2 rule: P = e4m3(2^t) and l sums the unquantised 2^t.
+// BF16: P = bf16(2^(t - m)) with m the running max, l unquantised.
+// out = O ds_v / l.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>

@@ -14,7 +14,9 @@
 //   grid-stride re-read in reverse order (the most recently read data is
 //   still in L2), x * qs in fp32, cvt.rn.satfinite to E4M3, packed 8-byte
 //   stores.  The last CTA to finish commits the ring and the scales.
-//   static: a single read-cast-store sweep over all three tensors.
+//   static (and ring-scale): a single read-cast-store sweep over all three
+//   tensors, writing packed [T, H, 128] codes or, for sequence-parallel
+//   attention, head-grouped [groups, T, H / groups, 128] send buffers.
 #include <cuda_runtime.h>
 
 #include "kernels.h"
