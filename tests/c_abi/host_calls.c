@@ -63,6 +63,28 @@ int main(void) {
   CHECK(fp8attn_varlen_fwd((const void*)16, (const void*)16, (const void*)16,
                            (const int32_t*)16, 1, 8, 8, 8, 64, (const float*)16, 0.0f,
                            (void*)16, (int32_t*)0, (void*)0) == FP8ATTN_ERR_UNSUPPORTED);
+  /* work schedules: the three named ones pass the checks (zero tokens), others
+   * are invalid */
+  CHECK(fp8attn_varlen_fwd_sched((const void*)0, (const void*)0, (const void*)0,
+                                 (const int32_t*)16, 1, 8, 0, 8, 128, (const float*)0, 0.0f,
+                                 FP8ATTN_P_LINEAR_LOG, FP8ATTN_SCHED_SPLIT, (void*)0,
+                                 (int32_t*)0, (void*)0) == FP8ATTN_OK);
+  CHECK(fp8attn_varlen_fwd_sched((const void*)0, (const void*)0, (const void*)0,
+                                 (const int32_t*)16, 1, 8, 0, 8, 128, (const float*)0, 0.0f,
+                                 FP8ATTN_P_EXP2, 7, (void*)0, (int32_t*)0,
+                                 (void*)0) == FP8ATTN_ERR_INVALID);
+  /* the grouped cast: DYNAMIC and a group count that does not divide the
+   * heads are refused before the context is touched */
+  CHECK(fp8attn_quantize_qkv_grouped((fp8attn_ctx*)0, 0, FP8ATTN_DYNAMIC, (const void*)16,
+                                     (const void*)16, (const void*)16, 1024, 128,
+                                     (const int32_t*)0, (const int32_t*)16, 1, 8, 8, 8, 128, 2,
+                                     (void*)16, (void*)16, (void*)16,
+                                     (void*)0) == FP8ATTN_ERR_INVALID);
+  CHECK(fp8attn_quantize_qkv_grouped((fp8attn_ctx*)0, 0, FP8ATTN_RING, (const void*)16,
+                                     (const void*)16, (const void*)16, 1024, 128,
+                                     (const int32_t*)0, (const int32_t*)16, 1, 8, 8, 8, 128, 3,
+                                     (void*)16, (void*)16, (void*)16,
+                                     (void*)0) == FP8ATTN_ERR_INVALID);
 
   /* the static scale map: parse (with the margin), format, apply_margin */
   {
