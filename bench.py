@@ -805,7 +805,9 @@ def run_ours(args):
 
     dyn = None if args.no_dynamic_quant else measure_dynamic_quant(dev, stream)
     peaks, src = load_peaks()
-    fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
+    fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16                      # burst
+    fp8_peak_sust = peaks.get("bf16_tflops_sustained",
+                              FALLBACK_PEAKS["bf16_tflops_sustained"]) * FP8_PER_BF16
 
     # this workload's error against unquantised fp64 attention, and the
     # attention time under the other P rule (outside the timed step)
@@ -874,11 +876,23 @@ def run_ours(args):
                           "fp8_speedup": bf16_s / fp8_alone_s},
             "err_vs_unquantized": err_uq,
             "quant_us": quant_s * 1e6, "quant_gbs": quant_gbs,
-            "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": fp8_peak,
-                         "unit": "TFLOP/s", "frac": attn_tflops / fp8_peak,
+            # the timed loop runs for about a second under the power cap, so
+            # its attention time is set against the sustained GEMM peak; the
+            # same kernel timed alone (20 launches, burst clocks) against the
+            # burst peak
+            "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": fp8_peak_sust,
+                         "unit": "TFLOP/s", "frac": attn_tflops / fp8_peak_sust,
+                         "peak_burst": fp8_peak, "frac_of_burst": attn_tflops / fp8_peak,
                          "traffic": attn_traffic, "traffic_source": attn_traffic_src,
                          "kernel": "attn_fwd_fp8_kernel",
-                         "peak_source": f"{src} bf16 burst x{FP8_PER_BF16:g} (fp8/bf16 nominal)"},
+                         "peak_source": f"{src} bf16 sustained x{FP8_PER_BF16:g} (fp8/bf16 "
+                                        f"nominal): timed inside the {K}-step loop"},
+            "attn_alone": {"attn_us": fp8_alone_s * 1e6,
+                           "attn_tflops": FLOPS_PER_STEP / fp8_alone_s / 1e12,
+                           "peak": fp8_peak,
+                           "frac": FLOPS_PER_STEP / fp8_alone_s / 1e12 / fp8_peak,
+                           "timing": "median of 20 launches", "l2": "flushed before each launch",
+                           "peak_source": f"{src} bf16 burst x{FP8_PER_BF16:g} (fp8/bf16 nominal)"},
             "quant_roofline": {"bound": "hbm", "achieved": quant_gbs, "peak": peaks["hbm_gbs"],
                                "unit": "GB/s", "frac": quant_gbs / peaks["hbm_gbs"],
                                "traffic": quant_traffic, "traffic_source": quant_traffic_src,
