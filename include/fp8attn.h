@@ -262,7 +262,9 @@ typedef enum {
  *     units would fill at most half of the SMs, each of those units runs as
  *     two CTAs of one tile each, so that the tiles fill that wave (a lone
  *     tile's blocks run faster than a CTA's two interleaved tiles); those
- *     CTAs form a second launch that starts as SMs free up.
+ *     CTAs form a second launch that starts as SMs free up.  When every
+ *     unit fits in that one wave (short sequences, few heads), all units
+ *     run that way, in one launch.
  *   FP8ATTN_SCHED_WHOLE: one CTA per unit.
  *   FP8ATTN_SCHED_SPLIT: every unit as two single-tile CTAs. */
 typedef enum {

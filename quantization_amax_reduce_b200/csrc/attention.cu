@@ -1031,7 +1031,8 @@ bool make_qkv_map(CUtensorMap* m, const void* base, int64_t T, int H, bool bf16)
 
 // How many of a launch's `units` (the last ones) run as two single-tile
 // CTAs each.  Auto: the units of a last wave that would fill at most half
-// of the SMs, so that their tiles fill that wave instead.
+// of the SMs, so that their tiles fill that wave instead; when all units fit
+// in that one wave, every unit.
 int64_t split_units(int64_t units, int schedule, int dev) {
   if (schedule == kSchedWhole) return 0;
   if (schedule == kSchedSplit) return units;
@@ -1048,7 +1049,7 @@ int64_t split_units(int64_t units, int schedule, int dev) {
     sms = n_sm[dev];
   }
   const int64_t tail = units % sms;
-  if (units <= sms || tail == 0 || 2 * tail > sms) return 0;
+  if (tail == 0 || 2 * tail > sms) return 0;
   return tail;
 }
 

@@ -3,7 +3,8 @@
 A work unit (256 query rows of one head of one sequence) is computed as two
 128-row tiles.  It runs either in one CTA that interleaves both tiles or as
 two CTAs of one tile each; the automatic schedule uses the second form for
-the units of a mostly empty last wave.  Every output row goes through the
+the units of a mostly empty last wave, and for all units when they fit in a
+single wave that fills at most half the SMs.  Every output row goes through the
 same key blocks, in the same order, under the same P rule either way, so the
 schedules must agree bit for bit, and each must match the oracle."""
 import numpy as np
@@ -37,7 +38,7 @@ def _run(q8, k8, v8, cu, ds, rule, schedule, scale=0.0):
 @pytest.mark.parametrize("rule,orule", RULES)
 @pytest.mark.parametrize("lens,H", [
     ([5000, 300, 8269], 2),       # 198 units: AUTO splits the last 50 on 148 SMs
-    ([129, 1, 257, 40], 3),       # single-tile CTAs whose second tile is empty
+    ([129, 1, 257, 40], 3),       # 24 units: AUTO splits them all; empty second tiles
     ([1000, 17], 40),             # 200 units, ragged sequences
 ])
 def test_schedules_agree_bit_for_bit_and_with_the_oracle(lens, H, rule, orule):
