@@ -496,11 +496,12 @@ def measure_per_config(dev, stream, p_rule, fp8_peak, flush):
         raise RuntimeError("device error in the per-workload runs")
 
     # How much of a static-scale step the separate quantisation launch takes
-    # at short and long sequences (the headroom a quantise-in-attention
-    # kernel could recover): one sequence of S tokens, 16 heads, N(0,1),
-    # static 224/198/210, each kernel timed alone after an L2 flush.
+    # at short and long sequences, and the same step as one launch with the
+    # cast inside the attention kernel (varlen_fwd_static, checked equal to
+    # the two launches): one sequence of S tokens, 16 heads, N(0,1), static
+    # 224/198/210, each timed after an L2 flush.
     share = []
-    for S_len in (256, 1024, 4096, 8192):
+    for S_len in (256, 512, 1024, 2048, 4096, 8192):
         g = torch.Generator(device=dev)
         g.manual_seed(1000 + S_len)
         src = [torch.randn(S_len, H, D, generator=g, device=dev).to(torch.bfloat16)
@@ -517,12 +518,27 @@ def measure_per_config(dev, stream, p_rule, fp8_peak, flush):
         def at():
             qar.varlen_fwd(*codes, cu_s, S_len, cs.descale_ptr(0), out=o, stream=stream,
                            p_rule=p_rule)
+        o2 = torch.empty_like(o)
+
+        def both():
+            qz()
+            at()
+
+        def fused():
+            cs.varlen_fwd_static(0, *src, cu_s, S_len, out=o2, stream=stream, p_rule=p_rule)
         qz()
         at()
+        fused()
+        torch.cuda.synchronize(dev)
+        if not torch.equal(o, o2):
+            raise RuntimeError(f"S={S_len}: the fused static call differs from cast + attention")
         tq = _time_launches(qz, dev, stream, 20, flush)
         ta = _time_launches(at, dev, stream, 20, flush)
+        tb = _time_launches(both, dev, stream, 20, flush)
+        tf = _time_launches(fused, dev, stream, 20, flush)
         share.append({"S": S_len, "heads": H, "quant_us": tq * 1e6, "attn_us": ta * 1e6,
-                      "quant_share": tq / (tq + ta)})
+                      "quant_share": tq / (tq + ta), "cast_then_attn_us": tb * 1e6,
+                      "fused_us": tf * 1e6, "fused_speedup": tb / tf})
     res["static_quant_share_by_length"] = share
     return res
 

@@ -254,6 +254,35 @@ typedef enum {
   FP8ATTN_P_EXP2 = 1
 } fp8attn_p_rule;
 
+/* Static-scale quantisation and FP8 attention in one launch: the result of
+ * fp8attn_quantize_qkv(ctx, layer, FP8ATTN_STATIC, q, k, v, tok_stride,
+ * head_stride, NULL, ...) followed by fp8attn_varlen_fwd on its codes with
+ * fp8attn_descale_ptr(ctx, layer), bit for bit, without the E4M3 copies of
+ * Q, K and V in device memory: the kernel casts Q as each CTA starts and K
+ * and V tile by tile between their TMA loads and the tensor-core products
+ * (vLLM FP8 ViT page, Notes: the separate quantisation launches are what
+ * costs small inputs their FP8 gain).
+ *   q, k, v: packed bf16 sources (one row per token, no padding); element
+ *     (t, h, d) at base + t*tok_stride + h*head_stride + d, strides in
+ *     elements, multiples of 8, head_stride >= head_dim and tok_stride >=
+ *     num_heads*head_stride (e.g. [T, H, 128], or an interleaved [T, 3, H,
+ *     128] projection output).  Other arguments as fp8attn_varlen_fwd_rule;
+ *     the work schedule is FP8ATTN_SCHED_AUTO.
+ * The layer's current scales become its static ones, as after the cast.
+ * Device-side errors (SEQLENS, TIMEOUT) go to the context's error word
+ * (fp8attn_get_error).  Errors: INVALID (no static scales for the layer,
+ * bad arguments), UNSUPPORTED (head_dim != 128, strides), CUDA.  With
+ * total_tokens == 0 nothing is launched.
+ * Speed: up to about 300 tokens a sequence this matches the two launches;
+ * beyond, every 256-query CTA of a head casts all of that head's K and V
+ * again, and the two launches are faster (2-3x at 2048-8192 tokens). */
+fp8attn_status fp8attn_varlen_fwd_static(fp8attn_ctx* ctx, int layer, const void* q,
+                                         const void* k, const void* v, int64_t tok_stride,
+                                         int64_t head_stride, const int32_t* d_cu_seqlens,
+                                         int batch, int max_seqlen, int64_t total_tokens,
+                                         int num_heads, int head_dim, float softmax_scale,
+                                         int p_rule, void* out, void* stream);
+
 /* How fp8attn_varlen_fwd_sched lays the work units (256 query rows of one
  * head of one sequence, computed as two 128-row tiles) on the GPU.  Each
  * output row is computed the same way under every schedule (same key

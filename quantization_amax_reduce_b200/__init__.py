@@ -94,6 +94,8 @@ def lib() -> ctypes.CDLL:
         "fp8attn_varlen_fwd_rule": (I, [P, P, P, P, I, I, I64, I, I, P, F, I, P, P, P]),
         "fp8attn_varlen_fwd_sched": (I, [P, P, P, P, I, I, I64, I, I, P, F, I, I, P, P, P]),
         "fp8attn_varlen_fwd_bf16": (I, [P, P, P, P, I, I, I64, I, I, F, P, P, P]),
+        "fp8attn_varlen_fwd_static": (I, [P, I, P, P, P, I64, I64, P, I, I, I64, I, I, F, I, P,
+                                          P]),
         "fp8attn_get_error": (I, [P, P]),
         "fp8attn_read_error_word": (I, [P, P]),
         "fp8attn_parse_selector": (I, [ctypes.c_char_p, I, U8P]),
@@ -277,6 +279,31 @@ class Context:
             _ptr(out[1]), _ptr(out[2]), ctypes.c_void_p(_stream(stream, q.device))),
             "fp8attn_quantize_qkv")
         return out[0], out[1], out[2]
+
+    def varlen_fwd_static(self, layer: int, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                          cu_seqlens, max_seqlen: int, *, softmax_scale: float = 0.0,
+                          total_tokens: Optional[int] = None, out: Optional[torch.Tensor] = None,
+                          stream=None, p_rule: int = P_LINEAR_LOG) -> torch.Tensor:
+        """Static-scale quantisation and FP8 attention in one launch: bit for
+        bit ``varlen_fwd(*quantize_qkv(layer, STATIC, q, k, v, ...), ...,
+        descale_ptr(layer))`` without the E4M3 copies in device memory.
+        Sources are packed bf16 [T, H, 128] or a strided view of that shape
+        (e.g. slices of a fused [T, 3, H, 128] projection); returns bf16
+        [T, H, 128].  Device-side errors go to the context (``get_error``)."""
+        if q.dim() != 3:
+            raise ValueError("sources are packed [T, H, 128] (no padded layout)")
+        H, tok_stride, head_stride, cu, B, total_tokens, _ = _qkv_source(
+            q, k, v, cu_seqlens, total_tokens, None)
+        n = int(total_tokens) * H * HEAD_DIM
+        if out is None:
+            out = torch.empty((total_tokens, H, HEAD_DIM), dtype=torch.bfloat16, device=q.device)
+        else:
+            _check_out(out, "out", torch.bfloat16, n, q.device)
+        _check(lib().fp8attn_varlen_fwd_static(
+            self._h, layer, _ptr(q), _ptr(k), _ptr(v), tok_stride, head_stride, _ptr(cu), B,
+            int(max_seqlen), int(total_tokens), H, HEAD_DIM, float(softmax_scale), int(p_rule),
+            _ptr(out), ctypes.c_void_p(_stream(stream, q.device))), "fp8attn_varlen_fwd_static")
+        return out
 
     def quantize_qkv_grouped(self, layer: int, mode: int, q: torch.Tensor, k: torch.Tensor,
                              v: torch.Tensor, cu_seqlens, max_seqlen: int, groups: int, *,

@@ -455,6 +455,52 @@ fp8attn_status fp8attn_varlen_fwd_sched(const void* q8, const void* k8, const vo
                        schedule);
 }
 
+fp8attn_status fp8attn_varlen_fwd_static(fp8attn_ctx* ctx, int layer, const void* q,
+                                         const void* k, const void* v, int64_t tok_stride,
+                                         int64_t head_stride, const int32_t* d_cu_seqlens,
+                                         int batch, int max_seqlen, int64_t total_tokens,
+                                         int num_heads, int head_dim, float softmax_scale,
+                                         int p_rule, void* out, void* stream) {
+  if (!layer_ok(ctx, layer) || !ctx->has_static[layer]) return FP8ATTN_ERR_INVALID;
+  if (p_rule != FP8ATTN_P_LINEAR_LOG && p_rule != FP8ATTN_P_EXP2) return FP8ATTN_ERR_INVALID;
+  fp8attn_status st = check_attention(q, k, v, d_cu_seqlens, batch, max_seqlen, total_tokens,
+                                      num_heads, head_dim, out);
+  if (st != FP8ATTN_OK || total_tokens == 0) return st;
+  if (!(softmax_scale >= 0.0f) || std::isinf(softmax_scale)) return FP8ATTN_ERR_INVALID;
+  // rows of heads of 128 channels, heads within a row, no overlap; strides in
+  // 16-byte units (the TMA map's rule)
+  if (tok_stride <= 0 || head_stride <= 0 || (tok_stride % 8) || (head_stride % 8) ||
+      head_stride < head_dim || tok_stride < static_cast<int64_t>(num_heads) * head_stride)
+    return FP8ATTN_ERR_UNSUPPORTED;
+  LayerState* ls = ctx->ls + layer;
+  AttnLaunch a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.cu = d_cu_seqlens;
+  a.batch = batch;
+  a.heads = num_heads;
+  a.max_seqlen = max_seqlen;
+  a.descale = ls->static_ds;
+  a.softmax_scale = softmax_scale == 0.0f ? 1.0f / std::sqrt(static_cast<float>(head_dim))
+                                          : softmax_scale;
+  a.out = out;
+  a.err = reinterpret_cast<int32_t*>(&ctx->gs->error);
+  a.bf16 = 0;
+  a.p_rule = p_rule == FP8ATTN_P_EXP2 ? kPRuleExp2 : kPRuleLinearLog;
+  a.schedule = kSchedAuto;
+  a.fused = 1;
+  a.tok_stride = tok_stride;
+  a.head_stride = head_stride;
+  a.qscale = ls->static_qs;
+  a.cur_qs = ls->qs;
+  a.cur_ds = ls->ds;
+  const cudaError_t e = launch_attention(a, total_tokens, as_stream(stream));
+  if (e != cudaSuccess) return FP8ATTN_ERR_CUDA;
+  g_launches.fetch_add(1);
+  return FP8ATTN_OK;
+}
+
 fp8attn_status fp8attn_selftest_qk_scores(const void* d_q8, const void* d_k8, int64_t tiles,
                                           float* d_scores, int32_t* d_error, void* stream) {
   if (!d_q8 || !d_k8 || !d_scores || tiles < 1 || tiles > 0x7FFFFFFF / 128)

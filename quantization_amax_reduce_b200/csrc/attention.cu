@@ -20,9 +20,14 @@
 // attn_fwd_bf16_kernel: P_i aliases the first 64 columns of S_i and PV
 // reads it from TMEM; S_i(j+1) is issued after PV_i(j).
 // attn_fwd_fp8_kernel: P_i goes to shared memory, so S_i(j+1) is computed
-// while the softmax still works on block j.  Its <rule, 1> instantiation
+// while the softmax still works on block j.  Its <rule, 1, *> instantiation
 // runs a unit as two CTAs of one tile each (the automatic schedule's fill
-// for a mostly empty last wave, launched behind the whole units).
+// for a mostly empty last wave, launched behind the whole units).  Its
+// <rule, *, 1> instantiation takes bf16 Q/K/V and casts them with the
+// layer's static scales inside the kernel (384 threads): every warp casts Q
+// (and, for a sequence of at most 512 keys, all of K and V) straight from
+// global memory before the roles start; longer sequences stream bf16 K/V
+// tiles through TMA staging that the TMA warp and warp 11 cast.
 //
 // P rule (pages silent; fixed here), per 128-key block: c = ds_q ds_k
 // softmax_scale log2(e), t = s c - r + 5 against a reference max r that
@@ -39,6 +44,7 @@
 
 #include <cstdint>
 #include <mutex>
+#include <type_traits>
 
 #include "kernels.h"
 #include "sm100_ptx.cuh"
@@ -82,6 +88,22 @@ struct AttnParams {
   __nv_bfloat16* out;
   int32_t* err;
 };
+
+// The FP8 kernel with the static cast inside (kFused) also takes the bf16
+// sources and their strides (elements), the cast scales and the layer's
+// current scales.
+struct AttnParamsFused : AttnParams {
+  const uint16_t* qsrc;
+  const uint16_t* ksrc;
+  const uint16_t* vsrc;
+  int64_t tok_stride, head_stride;
+  const float* qscale;
+  float* cur_qs;
+  float* cur_ds;
+};
+
+template <int kFused>
+using Fp8Params = typename std::conditional<kFused != 0, AttnParamsFused, AttnParams>::type;
 
 struct Barriers {
   uint64_t q_full;
@@ -482,6 +504,11 @@ struct Fp8Cfg {
   static constexpr int kStages = 3;
   static constexpr int kTile = 16384;   // 128 x 128 bytes
   static constexpr int kSmemBytes = (2 + 2 * kStages + 4) * kTile + 1024 + 1024;
+  // static cast inside the kernel: four tiles each for K and V, holding
+  // either a whole short sequence's E4M3 K and V (up to 512 keys), or two
+  // E4M3 stages plus one bf16 staging tile of 32 KB
+  static constexpr int kTilesFused = 4;
+  static constexpr int kSmemBytesFused = (2 + 2 * kTilesFused + 4) * kTile + 1024 + 1024;
 };
 
 // FP8 kernel warps: 0-7 softmax, 8 TMA producer, 9 and 10 MMA issuers for
@@ -489,40 +516,90 @@ struct Fp8Cfg {
 // streams and their barrier waits overlap instead of queueing behind each
 // other; each tile's MMAs still complete in issue order).
 constexpr int kThreadsFp8 = 352;
+// With the static cast inside the kernel, warp 11 joins the TMA warp in
+// casting the bf16 K and V tiles (each warp 64 rows of every tile).
+constexpr int kThreadsFp8Fused = 384;
+constexpr int kCastWarp = 11;
 
+template <int kTiles>   // K (and V) tiles held in shared memory
 struct Fp8Barriers {
   uint64_t q_full;
-  uint64_t k_full[Fp8Cfg::kStages];
-  uint64_t v_full[Fp8Cfg::kStages];
-  uint64_t k_empty[Fp8Cfg::kStages];   // the S products that read the K stage are done
-  uint64_t v_empty[Fp8Cfg::kStages];   // the PV products that read the V stage are done
+  uint64_t k_full[kTiles];
+  uint64_t v_full[kTiles];
+  uint64_t k_empty[kTiles];   // the S products that read the K stage are done
+  uint64_t v_empty[kTiles];   // the PV products that read the V stage are done
   uint64_t s_full[2];       // S_i of the current block computed
   uint64_t s_free[2];       // S_i loaded by the softmax (TMEM columns free)
   uint64_t p_full[2][2];    // [tile][P buffer] P_i written
   uint64_t pv_done[2][2];   // [tile][P buffer] PV_i that read that buffer done
   uint64_t v_tail;          // the last, partial V tile's rows past the sequence are zeroed
   uint64_t drain[2];
+  uint64_t stg_full[2];     // [K, V] bf16 staging tile landed (static cast inside)
+  uint64_t stg_empty[2];    // [K, V] both cast warps have read the staging tile
   uint32_t tmem_base;
   int abort_flag;
 };
 
+// 16 bf16 (two 16-byte vectors, channels in order) -> 16 E4M3 codes of
+// fl32(x * qs), round to nearest even, saturating: the static cast of the
+// quantisation kernel.
+__device__ __forceinline__ uint4 cast16_e4m3(uint4 a, uint4 b, float qs) {
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  const uint64_t qs2 = f2_pack(qs, qs);
+  uint32_t h[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float lo, hi;
+    f2_unpack(f2_mul(f2_pack(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u)),
+                     qs2),
+              lo, hi);
+    h[i] = cvt_e4m3x2(lo, hi);
+  }
+  return make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16),
+                    h[6] | (h[7] << 16));
+}
+
+// Cast rows [64 w, 64 w + 64) of a bf16 K or V tile staged by TMA (two
+// 128B-swizzled boxes of 64 channels) into the E4M3 tile the MMA reads
+// (128B-swizzled, 128 channels a row).  Lane l takes rows l and l + 32 of the
+// half, 16 channels at a time, so that each group of 8 lanes touches 8 rows
+// of one chunk (no bank conflicts on either side).
+__device__ __forceinline__ void cast_tile_half(const uint8_t* stg, uint8_t* dst, int w, int lane,
+                                               float qs) {
+#pragma unroll 4
+  for (int n = 0; n < 16; ++n) {
+    const int row = 64 * w + lane + 32 * (n & 1);
+    const int cp = n >> 1;                 // 16 channels: 16 * cp ..
+    const int c = 2 * (cp & 3);            // first 16-byte chunk in the bf16 box
+    const uint8_t* src = stg + (cp >> 2) * 16384 + row * 128;
+    const uint4 a = *reinterpret_cast<const uint4*>(src + ((c ^ (row & 7)) << 4));
+    const uint4 b = *reinterpret_cast<const uint4*>(src + (((c + 1) ^ (row & 7)) << 4));
+    *reinterpret_cast<uint4*>(dst + row * 128 + ((cp ^ (row & 7)) << 4)) = cast16_e4m3(a, b, qs);
+  }
+}
+
 // kSplit = 0: each CTA runs one work unit as two interleaved 128-row tiles.
 // kSplit = 1: each unit runs as two CTAs of one tile each.  The two are
 // separate instantiations so that each compiles with its tile count fixed.
-template <int kRule, int kSplit>
-__global__ void __launch_bounds__(kThreadsFp8, 1)
+// kFused = 1: Q, K and V arrive as bf16 and are cast with the static scales
+// inside the kernel (Q by all warps before the roles start, K and V tile by
+// tile by the TMA warp and warp 11 between the TMA loads and the MMAs), so
+// no E4M3 copy of the inputs goes through HBM.
+template <int kRule, int kSplit, int kFused>
+__global__ void __launch_bounds__(kFused ? kThreadsFp8Fused : kThreadsFp8, 1)
 attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, AttnParams p) {
+                    const __grid_constant__ CUtensorMap tm_v, Fp8Params<kFused> p) {
   using C = Fp8Cfg;
+  constexpr int kSt = kFused ? C::kTilesFused : C::kStages;   // K (and V) tiles in smem
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sq = smem;                                   // 2 Q tiles
   uint8_t* sk = smem + 2 * C::kTile;                    // kStages K tiles
-  uint8_t* sv = sk + C::kStages * C::kTile;             // kStages V tiles
-  uint8_t* sp = sv + C::kStages * C::kTile;             // P [tile][buffer]
-  Fp8Barriers& bars = *reinterpret_cast<Fp8Barriers*>(sp + 4 * C::kTile);
+  uint8_t* sv = sk + kSt * C::kTile;             // kStages V tiles
+  uint8_t* sp = sv + kSt * C::kTile;             // P [tile][buffer]
+  Fp8Barriers<kSt>& bars = *reinterpret_cast<Fp8Barriers<kSt>*>(sp + 4 * C::kTile);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -532,6 +609,14 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
   if (kSplit == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // work unit = (query block of 256 rows, head, sequence)
   const int cta = static_cast<int>(blockIdx.x);
+  if constexpr (kFused != 0) {
+    if (p.unit0 == 0 && cta == 0 && threadIdx.x < 3) {
+      // the cast scales become the layer's current scales (as after a cast
+      // launch); one CTA of the call writes them, whatever its unit holds
+      p.cur_qs[threadIdx.x] = __ldg(p.qscale + threadIdx.x);
+      p.cur_ds[threadIdx.x] = __ldg(p.descale + threadIdx.x);
+    }
+  }
   constexpr int ntiles = kSplit ? 1 : 2;
   const int unit = p.unit0 + (kSplit ? (cta >> 1) : cta);
   const int sub = kSplit ? (cta & 1) : 0;
@@ -554,12 +639,18 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
     return;
   }
   const int nkv = (len + 127) / 128;
+  // kFused: a sequence of up to kTilesFused key blocks is cast whole into
+  // shared memory by all warps up front; longer ones stream through two
+  // E4M3 stages, tiles 2-3 of each buffer staging the bf16 tile
+  const bool resident = kFused && nkv <= C::kTilesFused;
+  const int nst = kFused ? (resident ? C::kTilesFused : 2) : C::kStages;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars.q_full, 1);
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&bars.k_full[s], 1);
-      mbar_init(&bars.v_full[s], 1);
+    for (int s = 0; s < kSt; ++s) {
+      // kFused: filled by the two cast warps (one elected arrive each)
+      mbar_init(&bars.k_full[s], kFused ? 2 : 1);
+      mbar_init(&bars.v_full[s], kFused ? 2 : 1);
       mbar_init(&bars.k_empty[s], ntiles);   // one commit per active MMA warp
       mbar_init(&bars.v_empty[s], ntiles);
     }
@@ -574,6 +665,10 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(&bars.v_tail, 1);
     mbar_init(&bars.drain[0], 1);
     mbar_init(&bars.drain[1], 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars.stg_full[t], 1);
+      mbar_init(&bars.stg_empty[t], 2);
+    }
     bars.abort_flag = 0;
     fence_mbar_init();
   }
@@ -587,7 +682,150 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t tmem = bars.tmem_base;
   const volatile int* abort_flag = &bars.abort_flag;
 
-  if (warp == kTmaWarp) {
+  if constexpr (kFused != 0) {
+    if (!resident && warp == kTmaWarp && lane == 0) {
+      // the first K and V tiles start landing (as bf16, in tiles 2-3 of the
+      // K and V buffers) while Q is cast
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      for (int t = 0; t < 2; ++t) {
+        const CUtensorMap* m = t ? &tm_v : &tm_k;
+        uint8_t* stg = (t ? sv : sk) + 2 * C::kTile;
+        mbar_expect_tx(&bars.stg_full[t], 2 * C::kTile);
+        tma_load_3d(stg, m, &bars.stg_full[t], 0, h, seq0);
+        tma_load_3d(stg + C::kTile, m, &bars.stg_full[t], 64, h, seq0);
+      }
+    }
+    // Q (and, for a resident sequence, K and V): every thread casts 32-byte
+    // pieces (16 channels of a row) straight from global memory, loading
+    // kBatch pieces before casting any (the loads' latency overlaps); rows
+    // past the sequence become zeros.  Item order: Q rows, then K, V tiles.
+    constexpr int kBatch = 8;
+    const int nq = ntiles * 128 * 8;
+    const int nitems = nq + (resident ? nkv * 2 * 1024 : 0);
+    const int tid = static_cast<int>(threadIdx.x);
+    for (int it0 = tid; it0 < nitems; it0 += kBatch * kThreadsFp8Fused) {
+      uint4 xa[kBatch], xb[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int it = it0 + u * kThreadsFp8Fused;
+        xa[u] = xb[u] = make_uint4(0u, 0u, 0u, 0u);
+        int row, t;
+        if (it < nq) {
+          row = q0 + (it >> 3);
+          t = 0;
+        } else {
+          const int x = it - nq;
+          row = 128 * (x >> 11) + ((x >> 3) & 127);
+          t = 1 + ((x >> 10) & 1);
+        }
+        if (it < nitems && row < len) {
+          const uint16_t* base = t == 0 ? p.qsrc : t == 1 ? p.ksrc : p.vsrc;
+          const uint4* src = reinterpret_cast<const uint4*>(
+              base + static_cast<int64_t>(seq0 + row) * p.tok_stride +
+              static_cast<int64_t>(h) * p.head_stride + 16 * (it & 7));
+          xa[u] = __ldg(src);
+          xb[u] = __ldg(src + 1);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int it = it0 + u * kThreadsFp8Fused;
+        if (it >= nitems) break;
+        const int cp = it & 7;
+        int r, row, t;
+        uint8_t* dst;
+        if (it < nq) {
+          r = it >> 3;
+          row = q0 + r;
+          t = 0;
+          dst = sq + (r >> 7) * C::kTile;
+        } else {
+          const int x = it - nq;
+          const int tj = x >> 10;    // 2 j + (0 K, 1 V)
+          r = (x >> 3) & 127;
+          row = 128 * (tj >> 1) + r;
+          t = 1 + (tj & 1);
+          dst = (t == 1 ? sk : sv) + (tj >> 1) * C::kTile;
+        }
+        const int rr = r & 127;
+        const uint4 codes = row < len ? cast16_e4m3(xa[u], xb[u], __ldg(p.qscale + t))
+                                      : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(dst + rr * 128 + ((cp ^ (rr & 7)) << 4)) = codes;
+      }
+    }
+    fence_proxy_async();
+    __syncthreads();
+    if (resident && threadIdx.x == 0) {
+      // every K and V tile is in place (two arrivals: the full barriers
+      // count the two cast warps of the streaming form)
+      for (int j = 0; j < nkv; ++j)
+        for (int a = 0; a < 2; ++a) {
+          mbar_arrive(&bars.k_full[j]);
+          mbar_arrive(&bars.v_full[j]);
+        }
+    }
+  }
+
+  bool cast_role = false;
+  if constexpr (kFused != 0) {
+    if (warp == kTmaWarp || warp == kCastWarp) {
+    cast_role = true;
+    if (!resident) {
+    // ------------------------------------------------------------ K/V cast
+    // Tile order K_0, V_0, K_1, V_1, ...: staging buffer 0 holds K, 1 holds
+    // V.  Both warps cast their 64 rows of a staged tile into the free E4M3
+    // stage, then arrive on its full barrier and on the staging buffer's
+    // empty barrier; the TMA warp's lane 0 then loads the next tile of that
+    // kind into the staging buffer.
+    const int w = warp == kTmaWarp ? 0 : 1;
+    const bool issuer = warp == kTmaWarp;
+    const float qsk = __ldg(p.qscale + 1), qsv = __ldg(p.qscale + 2);
+    int issued[2] = {1, 1};   // tiles loaded into each staging buffer
+    bool ok = true;
+    for (int j = 0; j < nkv && ok; ++j) {
+      const int st = j % nst;
+      for (int t = 0; t < 2; ++t) {
+        uint8_t* buf = t ? sv : sk;
+        ok = mbar_wait(&bars.stg_full[t], j & 1, abort_flag);
+        if (ok && j >= nst)
+          ok = mbar_wait(t ? &bars.v_empty[st] : &bars.k_empty[st], ((j / nst) - 1) & 1, abort_flag);
+        if (!ok) break;
+        cast_tile_half(buf + 2 * C::kTile, buf + st * C::kTile, w, lane, t ? qsv : qsk);
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(t ? &bars.v_full[st] : &bars.k_full[st]);
+          mbar_arrive(&bars.stg_empty[t]);
+        }
+        if (issuer && j + 1 < nkv) {
+          // both warps are done reading: the next tile of this kind may land
+          ok = mbar_wait(&bars.stg_empty[t], j & 1, abort_flag);
+          if (!ok) break;
+          if (lane == 0) {
+            const CUtensorMap* m = t ? &tm_v : &tm_k;
+            mbar_expect_tx(&bars.stg_full[t], 2 * C::kTile);
+            tma_load_3d(buf + 2 * C::kTile, m, &bars.stg_full[t], 0, h, seq0 + 128 * (j + 1));
+            tma_load_3d(buf + 3 * C::kTile, m, &bars.stg_full[t], 64, h, seq0 + 128 * (j + 1));
+          }
+          ++issued[t];
+          __syncwarp();
+        }
+      }
+    }
+    if (!ok && lane == 0) note_error(p, bars, kErrTimeout);
+    if (issuer) {
+      // no copy may still be landing when the CTA leaves: wait for the last
+      // tile loaded into each staging buffer (completed phases pass at once)
+      for (int t = 0; t < 2; ++t)
+        mbar_wait(&bars.stg_full[t], (issued[t] - 1) & 1, nullptr);
+    }
+    }
+    }
+  }
+  if (cast_role) {
+    // (done above)
+  } else if (warp == kTmaWarp) {
     // ------------------------------------------------------------ producer
     const bool leader = lane == 0;
     if (leader) {
@@ -610,8 +848,8 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
     while (jv < nkv) {
       bool progressed = false;
       if (jk < nkv) {
-        const int st = jk % C::kStages;
-        if (jk < C::kStages || mbar_test_now(&bars.k_empty[st], ((jk / C::kStages) - 1) & 1)) {
+        const int st = jk % kSt;
+        if (jk < kSt || mbar_test_now(&bars.k_empty[st], ((jk / kSt) - 1) & 1)) {
           if (leader) {
             mbar_expect_tx(&bars.k_full[st], C::kTile);
             tma_load_3d(sk + st * C::kTile, &tm_k, &bars.k_full[st], 0, h, seq0 + 128 * jk);
@@ -621,8 +859,8 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
       }
       if (jv < jk) {
-        const int st = jv % C::kStages;
-        if (jv < C::kStages || mbar_test_now(&bars.v_empty[st], ((jv / C::kStages) - 1) & 1)) {
+        const int st = jv % kSt;
+        if (jv < kSt || mbar_test_now(&bars.v_empty[st], ((jv / kSt) - 1) & 1)) {
           if (leader) {
             mbar_expect_tx(&bars.v_full[st], C::kTile);
             tma_load_3d(sv + st * C::kTile, &tm_v, &bars.v_full[st], 0, h, seq0 + 128 * jv);
@@ -644,10 +882,10 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     if (!ok && leader) note_error(p, bars, kErrTimeout);
     // make sure no copy is still landing when the CTA leaves
-    for (int j = (jk > C::kStages ? jk - C::kStages : 0); j < jk; ++j)
-      mbar_wait(&bars.k_full[j % C::kStages], (j / C::kStages) & 1, nullptr);
-    for (int j = (jv > C::kStages ? jv - C::kStages : 0); j < jv; ++j)
-      mbar_wait(&bars.v_full[j % C::kStages], (j / C::kStages) & 1, nullptr);
+    for (int j = (jk > kSt ? jk - kSt : 0); j < jk; ++j)
+      mbar_wait(&bars.k_full[j % kSt], (j / kSt) & 1, nullptr);
+    for (int j = (jv > kSt ? jv - kSt : 0); j < jv; ++j)
+      mbar_wait(&bars.v_full[j % kSt], (j / kSt) & 1, nullptr);
     mbar_wait(&bars.q_full, 0, nullptr);
   } else if ((warp == kMmaWarp || warp == kMmaWarp + 1) && warp - kMmaWarp < ntiles) {
     // ------------------------------------------------------------ MMA issuers
@@ -659,11 +897,11 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
     const uint64_t dk0 = make_sdesc_sw128(smem_u32(sk), 16, 1024);
     const uint64_t dv0 = make_sdesc_sw128(smem_u32(sv), 16384, 1024);
     const uint64_t dp0 = make_sdesc_sw128(smem_u32(sp), 16, 1024);
-    constexpr uint32_t kStep = C::kTile >> 4;
+    constexpr uint32_t nstep = C::kTile >> 4;
     const uint32_t tS = tmem + 128 * i, tO = tmem + 256 + 128 * i;
     auto issue_s = [&](int j) {
       uint64_t ad[4], bd[4];
-      const uint64_t dk = dk0 + static_cast<uint64_t>((j % C::kStages) * kStep);
+      const uint64_t dk = dk0 + static_cast<uint64_t>((j % nst) * nstep);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         ad[kk] = dq + 2 * kk;   // 32 bytes of K per MMA
@@ -674,14 +912,14 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tS, ad[kk], bd[kk], id_qk, kk > 0);
         mma_commit(&bars.s_full[i]);
         // the K stage is free once both tiles' S products of block j are done
-        mma_commit(&bars.k_empty[j % C::kStages]);
+        mma_commit(&bars.k_empty[j % nst]);
       }
       __syncwarp();
     };
     auto issue_pv = [&](int j) {
       uint64_t ad[4], bd[4];
-      const uint64_t dp = dp0 + static_cast<uint64_t>((2 * i + (j & 1)) * kStep);
-      const uint64_t dv = dv0 + static_cast<uint64_t>((j % C::kStages) * kStep);
+      const uint64_t dp = dp0 + static_cast<uint64_t>((2 * i + (j & 1)) * nstep);
+      const uint64_t dv = dv0 + static_cast<uint64_t>((j % nst) * nstep);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         ad[kk] = dp + 2 * kk;          // P is K-major: 32 keys per MMA
@@ -692,27 +930,28 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tO, ad[kk], bd[kk], id_pv, kk > 0 ? 1u : acc0);
         mma_commit(&bars.pv_done[i][j & 1]);
-        mma_commit(&bars.v_empty[j % C::kStages]);
+        mma_commit(&bars.v_empty[j % nst]);
       }
       __syncwarp();
     };
-    bool ok = mbar_wait(&bars.q_full, 0, abort_flag) && mbar_wait(&bars.k_full[0], 0, abort_flag);
+    bool ok = (kFused || mbar_wait(&bars.q_full, 0, abort_flag)) &&
+              mbar_wait(&bars.k_full[0], 0, abort_flag);
     if (ok) {
       tc_fence_after();
       issue_s(0);
     }
     for (int j = 0; j < nkv && ok; ++j) {
-      const int st = j % C::kStages;
+      const int st = j % nst;
       if (j + 1 < nkv) {
-        const int st1 = (j + 1) % C::kStages;
+        const int st1 = (j + 1) % nst;
         // S_i's TMEM columns are free once the softmax has loaded block j
-        ok = mbar_wait(&bars.k_full[st1], ((j + 1) / C::kStages) & 1, abort_flag) &&
+        ok = mbar_wait(&bars.k_full[st1], ((j + 1) / nst) & 1, abort_flag) &&
              mbar_wait(&bars.s_free[i], j & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
         issue_s(j + 1);
       }
-      ok = mbar_wait(&bars.v_full[st], (j / C::kStages) & 1, abort_flag);
+      ok = mbar_wait(&bars.v_full[st], (j / nst) & 1, abort_flag);
       if (ok && j + 1 == nkv && (len & 127)) {
         // tile 0's warp zeroes the rows past the sequence; tile 1's waits for it
         if (i == 0) {
@@ -1029,6 +1268,22 @@ bool make_qkv_map(CUtensorMap* m, const void* base, int64_t T, int H, bool bf16)
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 source [T rows][H heads][128] with row and head strides in elements
+// (multiples of 8), 64-channel boxes of 128 rows, 128B swizzle.
+bool make_bf16_src_map(CUtensorMap* m, const void* base, int64_t T, int H, int64_t tok_stride,
+                       int64_t head_stride) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_stride) * 2,
+                           static_cast<cuuint64_t>(tok_stride) * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // How many of a launch's `units` (the last ones) run as two single-tile
 // CTAs each.  Auto: the units of a last wave that would fill at most half
 // of the SMs, so that their tiles fill that wave instead; when all units fit
@@ -1055,16 +1310,30 @@ int64_t split_units(int64_t units, int schedule, int dev) {
 
 // Launches `n_units` work units from `unit0` on (kSplit: two single-tile CTAs
 // per unit; `behind`: programmatic launch behind the previous kernel).
-template <bool kFp8, int kRule, int kSplit>
+template <bool kFp8, int kRule, int kSplit, int kFused>
 cudaError_t launch_attention_t(const AttnLaunch& a, int64_t T, cudaStream_t stream,
                                int64_t unit0, int64_t n_units, bool behind) {
   CUtensorMap mq, mk, mv;
-  if (!make_qkv_map(&mq, a.q, T, a.heads, !kFp8) || !make_qkv_map(&mk, a.k, T, a.heads, !kFp8) ||
-      !make_qkv_map(&mv, a.v, T, a.heads, !kFp8))
+  if (kFused) {
+    // K and V through TMA as bf16; Q is read by the CTA's threads (map unused)
+    if (!make_bf16_src_map(&mk, a.k, T, a.heads, a.tok_stride, a.head_stride) ||
+        !make_bf16_src_map(&mv, a.v, T, a.heads, a.tok_stride, a.head_stride))
+      return cudaErrorInvalidValue;
+    mq = mk;
+  } else if (!make_qkv_map(&mq, a.q, T, a.heads, !kFp8) ||
+             !make_qkv_map(&mk, a.k, T, a.heads, !kFp8) ||
+             !make_qkv_map(&mv, a.v, T, a.heads, !kFp8)) {
     return cudaErrorInvalidValue;
+  }
   // FP8 runs the P-in-shared-memory kernel; BF16 keeps P in TMEM
-  auto kernel = kFp8 ? attn_fwd_fp8_kernel<kRule, kSplit> : attn_fwd_bf16_kernel;
-  const int smem_bytes = kFp8 ? Fp8Cfg::kSmemBytes : Bf16Cfg::kSmemBytes;
+  using Prm = typename std::conditional<kFp8, Fp8Params<kFused>, AttnParams>::type;
+  void (*kernel)(CUtensorMap, CUtensorMap, CUtensorMap, Prm);
+  if constexpr (kFp8)
+    kernel = attn_fwd_fp8_kernel<kRule, kSplit, kFused>;
+  else
+    kernel = attn_fwd_bf16_kernel;
+  const int smem_bytes =
+      kFp8 ? (kFused ? Fp8Cfg::kSmemBytesFused : Fp8Cfg::kSmemBytes) : Bf16Cfg::kSmemBytes;
   // the shared-memory opt-in is a per-device function attribute: set it once
   // for each device this process launches on
   static std::mutex mu;
@@ -1093,10 +1362,22 @@ cudaError_t launch_attention_t(const AttnLaunch& a, int64_t T, cudaStream_t stre
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.err = a.err;
   p.unit0 = static_cast<int>(unit0);
+  Prm prm;
+  static_cast<AttnParams&>(prm) = p;
+  if constexpr (kFp8 && kFused != 0) {
+    prm.qsrc = static_cast<const uint16_t*>(a.q);
+    prm.ksrc = static_cast<const uint16_t*>(a.k);
+    prm.vsrc = static_cast<const uint16_t*>(a.v);
+    prm.tok_stride = a.tok_stride;
+    prm.head_stride = a.head_stride;
+    prm.qscale = a.qscale;
+    prm.cur_qs = a.cur_qs;
+    prm.cur_ds = a.cur_ds;
+  }
   const int64_t grid = kSplit ? 2 * n_units : n_units;
-  const int threads = kFp8 ? kThreadsFp8 : kThreadsAttn;
+  const int threads = kFp8 ? (kFused ? kThreadsFp8Fused : kThreadsFp8) : kThreadsAttn;
   if (!behind) {
-    kernel<<<static_cast<unsigned>(grid), threads, smem_bytes, stream>>>(mq, mk, mv, p);
+    kernel<<<static_cast<unsigned>(grid), threads, smem_bytes, stream>>>(mq, mk, mv, prm);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg = {};
@@ -1109,7 +1390,7 @@ cudaError_t launch_attention_t(const AttnLaunch& a, int64_t T, cudaStream_t stre
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, mq, mk, mv, p);
+  return cudaLaunchKernelEx(&cfg, kernel, mq, mk, mv, prm);
 }
 
 }  // namespace
@@ -1128,31 +1409,36 @@ cudaError_t launch_qk_scores_probe(const void* q8, const void* k8, int64_t tiles
   return cudaGetLastError();
 }
 
-template <int kRule>
+template <int kRule, int kFused>
 cudaError_t launch_fp8(const AttnLaunch& a, int64_t T, cudaStream_t stream, int64_t units,
                        int64_t split) {
   // whole units first, then the split units' single-tile CTAs behind them
   const int64_t whole = units - split;
   if (whole > 0) {
-    cudaError_t e = launch_attention_t<true, kRule, 0>(a, T, stream, 0, whole, false);
+    cudaError_t e = launch_attention_t<true, kRule, 0, kFused>(a, T, stream, 0, whole, false);
     if (e != cudaSuccess || split == 0) return e;
     note_launch();   // the caller counts one launch
   }
-  return launch_attention_t<true, kRule, 1>(a, T, stream, whole, split, whole > 0);
+  return launch_attention_t<true, kRule, 1, kFused>(a, T, stream, whole, split, whole > 0);
 }
 
 cudaError_t launch_attention(const AttnLaunch& a, int64_t total_tokens, cudaStream_t stream) {
   const int64_t units = static_cast<int64_t>((a.max_seqlen + 255) / 256) * a.heads * a.batch;
   if (units <= 0) return cudaSuccess;
   if (units > 0x3FFFFFFF) return cudaErrorInvalidConfiguration;
-  if (a.bf16) return launch_attention_t<false, kPRuleExp2, 0>(a, total_tokens, stream, 0, units, false);
+  if (a.bf16)
+    return launch_attention_t<false, kPRuleExp2, 0, 0>(a, total_tokens, stream, 0, units, false);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   const int64_t split = split_units(units, a.schedule, dev);
-  return a.p_rule == kPRuleExp2 ? launch_fp8<kPRuleExp2>(a, total_tokens, stream, units, split)
-                                : launch_fp8<kPRuleLinearLog>(a, total_tokens, stream, units, split);
+  if (a.fused)
+    return a.p_rule == kPRuleExp2
+               ? launch_fp8<kPRuleExp2, 1>(a, total_tokens, stream, units, split)
+               : launch_fp8<kPRuleLinearLog, 1>(a, total_tokens, stream, units, split);
+  return a.p_rule == kPRuleExp2 ? launch_fp8<kPRuleExp2, 0>(a, total_tokens, stream, units, split)
+                                : launch_fp8<kPRuleLinearLog, 0>(a, total_tokens, stream, units, split);
 }
 
 

@@ -48,6 +48,15 @@ struct AttnLaunch {
   int bf16;                      // 1 = native bf16 inputs (skip-layer path)
   int p_rule;                    // FP8 only: kPRuleLinearLog or kPRuleExp2
   int schedule;                  // FP8 only: kSchedAuto, kSchedWhole or kSchedSplit
+  // FP8 with the static cast inside the kernel: q, k, v are bf16 sources
+  // (element (t, h, d) at base + t * tok_stride + h * head_stride + d), cast
+  // with qscale {qs_q, qs_k, qs_v}; the first CTA copies qscale and descale
+  // to cur_qs / cur_ds (the layer's current scales)
+  int fused = 0;
+  int64_t tok_stride = 0, head_stride = 0;
+  const float* qscale = nullptr;
+  float* cur_qs = nullptr;
+  float* cur_ds = nullptr;
 };
 
 // P rules of the FP8 kernel (the values of fp8attn_p_rule in fp8attn.h).

@@ -85,6 +85,12 @@ int main(void) {
                                      (const int32_t*)0, (const int32_t*)16, 1, 8, 8, 8, 128, 3,
                                      (void*)16, (void*)16, (void*)16,
                                      (void*)0) == FP8ATTN_ERR_INVALID);
+  /* the static cast inside attention: a missing context is refused before
+   * anything else is looked at */
+  CHECK(fp8attn_varlen_fwd_static((fp8attn_ctx*)0, 0, (const void*)16, (const void*)16,
+                                  (const void*)16, 1024, 128, (const int32_t*)16, 1, 8, 8, 8,
+                                  128, 0.0f, FP8ATTN_P_LINEAR_LOG, (void*)16,
+                                  (void*)0) == FP8ATTN_ERR_INVALID);
 
   /* the static scale map: parse (with the margin), format, apply_margin */
   {

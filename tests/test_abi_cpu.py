@@ -116,6 +116,10 @@ def test_host_argument_checks_need_no_gpu(L):
     assert L.fp8attn_selftest_bounded_waits(ctypes.c_uint64(0), ctypes.byref(n), None) == 1
     assert L.fp8attn_selftest_bounded_waits(ctypes.c_uint64(2 * 10**9), ctypes.byref(n), None) == 1
     assert L.fp8attn_selftest_bounded_waits(ctypes.c_uint64(10**6), None, None) == 1
+    # the static cast inside attention: no context -> INVALID, before any
+    # other argument is read
+    assert L.fp8attn_varlen_fwd_static(None, 0, P(16), P(16), P(16), 1024, 128, P(16), 1, 8, 8,
+                                       8, 128, 0.0, 0, P(16), None) == 1
     # the grouped cast: STATIC / RING only, groups dividing the heads, checked
     # before any CUDA call (mode DYNAMIC = 0, STATIC = 1, RING = 3)
     g = (P(16), P(16), P(16), 1024, 128, None, P(16), 1, 8, 8, 8, 128)
