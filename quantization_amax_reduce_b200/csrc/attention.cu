@@ -767,64 +767,62 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   }
 
+  // ------------------------------------------------------------ K/V cast
+  // Tile order K_0, V_0, K_1, V_1, ...: staging buffer 0 holds K, 1 holds
+  // V.  Both warps cast their 64 rows of a staged tile into the free E4M3
+  // stage, then arrive on its full barrier and on the staging buffer's
+  // empty barrier; the TMA warp's lane 0 then loads the next tile of that
+  // kind into the staging buffer.
   bool cast_role = false;
   if constexpr (kFused != 0) {
-    if (warp == kTmaWarp || warp == kCastWarp) {
-    cast_role = true;
-    if (!resident) {
-    // ------------------------------------------------------------ K/V cast
-    // Tile order K_0, V_0, K_1, V_1, ...: staging buffer 0 holds K, 1 holds
-    // V.  Both warps cast their 64 rows of a staged tile into the free E4M3
-    // stage, then arrive on its full barrier and on the staging buffer's
-    // empty barrier; the TMA warp's lane 0 then loads the next tile of that
-    // kind into the staging buffer.
-    const int w = warp == kTmaWarp ? 0 : 1;
-    const bool issuer = warp == kTmaWarp;
-    const float qsk = __ldg(p.qscale + 1), qsv = __ldg(p.qscale + 2);
-    int issued[2] = {1, 1};   // tiles loaded into each staging buffer
-    bool ok = true;
-    for (int j = 0; j < nkv && ok; ++j) {
-      const int st = j % nst;
-      for (int t = 0; t < 2; ++t) {
-        uint8_t* buf = t ? sv : sk;
-        ok = mbar_wait(&bars.stg_full[t], j & 1, abort_flag);
-        if (ok && j >= nst)
-          ok = mbar_wait(t ? &bars.v_empty[st] : &bars.k_empty[st], ((j / nst) - 1) & 1, abort_flag);
-        if (!ok) break;
-        cast_tile_half(buf + 2 * C::kTile, buf + st * C::kTile, w, lane, t ? qsv : qsk);
-        fence_proxy_async();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(t ? &bars.v_full[st] : &bars.k_full[st]);
-          mbar_arrive(&bars.stg_empty[t]);
-        }
-        if (issuer && j + 1 < nkv) {
-          // both warps are done reading: the next tile of this kind may land
-          ok = mbar_wait(&bars.stg_empty[t], j & 1, abort_flag);
+    cast_role = warp == kTmaWarp || warp == kCastWarp;
+    if (cast_role && !resident) {
+      const int w = warp == kTmaWarp ? 0 : 1;
+      const bool issuer = warp == kTmaWarp;
+      const float qsk = __ldg(p.qscale + 1), qsv = __ldg(p.qscale + 2);
+      int issued[2] = {1, 1};   // tiles loaded into each staging buffer
+      bool ok = true;
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int st = j % nst;
+        for (int t = 0; t < 2; ++t) {
+          uint8_t* buf = t ? sv : sk;
+          ok = mbar_wait(&bars.stg_full[t], j & 1, abort_flag);
+          if (ok && j >= nst)
+            ok = mbar_wait(t ? &bars.v_empty[st] : &bars.k_empty[st], ((j / nst) - 1) & 1, abort_flag);
           if (!ok) break;
-          if (lane == 0) {
-            const CUtensorMap* m = t ? &tm_v : &tm_k;
-            mbar_expect_tx(&bars.stg_full[t], 2 * C::kTile);
-            tma_load_3d(buf + 2 * C::kTile, m, &bars.stg_full[t], 0, h, seq0 + 128 * (j + 1));
-            tma_load_3d(buf + 3 * C::kTile, m, &bars.stg_full[t], 64, h, seq0 + 128 * (j + 1));
-          }
-          ++issued[t];
+          cast_tile_half(buf + 2 * C::kTile, buf + st * C::kTile, w, lane, t ? qsv : qsk);
+          fence_proxy_async();
           __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(t ? &bars.v_full[st] : &bars.k_full[st]);
+            mbar_arrive(&bars.stg_empty[t]);
+          }
+          if (issuer && j + 1 < nkv) {
+            // both warps are done reading: the next tile of this kind may land
+            ok = mbar_wait(&bars.stg_empty[t], j & 1, abort_flag);
+            if (!ok) break;
+            if (lane == 0) {
+              const CUtensorMap* m = t ? &tm_v : &tm_k;
+              mbar_expect_tx(&bars.stg_full[t], 2 * C::kTile);
+              tma_load_3d(buf + 2 * C::kTile, m, &bars.stg_full[t], 0, h, seq0 + 128 * (j + 1));
+              tma_load_3d(buf + 3 * C::kTile, m, &bars.stg_full[t], 64, h, seq0 + 128 * (j + 1));
+            }
+            ++issued[t];
+            __syncwarp();
+          }
         }
       }
-    }
-    if (!ok && lane == 0) note_error(p, bars, kErrTimeout);
-    if (issuer) {
-      // no copy may still be landing when the CTA leaves: wait for the last
-      // tile loaded into each staging buffer (completed phases pass at once)
-      for (int t = 0; t < 2; ++t)
-        mbar_wait(&bars.stg_full[t], (issued[t] - 1) & 1, nullptr);
-    }
-    }
+      if (!ok && lane == 0) note_error(p, bars, kErrTimeout);
+      if (issuer) {
+        // no copy may still be landing when the CTA leaves: wait for the last
+        // tile loaded into each staging buffer (completed phases pass at once)
+        for (int t = 0; t < 2; ++t)
+          mbar_wait(&bars.stg_full[t], (issued[t] - 1) & 1, nullptr);
+      }
     }
   }
   if (cast_role) {
-    // (done above)
+    // the K/V cast above (static cast inside the kernel, streaming form)
   } else if (warp == kTmaWarp) {
     // ------------------------------------------------------------ producer
     const bool leader = lane == 0;
