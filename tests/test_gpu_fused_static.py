@@ -151,3 +151,18 @@ def test_fused_needs_static_scales_and_packed_rows():
     with pytest.raises(qar.FP8AttnError):
         ctx.varlen_fwd_static(1, over, over, over, cu_d, 10)
     assert ctx.get_error() == 0
+
+
+def test_fused_bad_cu_seqlens_sets_the_context_error():
+    """A decreasing cu_seqlens: the broken sequence writes nothing and the
+    context's error word reports SEQLENS; the valid one is computed."""
+    cu = torch.tensor([0, 100, 50], dtype=torch.int32, device=DEV)
+    q = torch.zeros(300, 1, 128, dtype=torch.bfloat16, device=DEV)
+    out = torch.full((300, 1, 128), 7.0, dtype=torch.bfloat16, device=DEV)
+    ctx = qar.Context(1)
+    ctx.set_static_scales(0, *BOUNDS)
+    ctx.varlen_fwd_static(0, q, q, q, cu, 300, out=out)
+    assert ctx.get_error() == 6
+    assert (out[100:] == 7.0).all()
+    assert (out[:100] == 0.0).all()
+    assert ctx.get_error() == 0
