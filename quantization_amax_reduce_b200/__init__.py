@@ -294,15 +294,21 @@ class Context:
             raise ValueError("sources are packed [T, H, 128] (no padded layout)")
         H, tok_stride, head_stride, cu, B, total_tokens, _ = _qkv_source(
             q, k, v, cu_seqlens, total_tokens, None)
+        dev = self.workspace.device          # the context's concrete device
+        if q.device != dev or cu.device != dev:
+            # the kernel reads the context's scales from its device workspace
+            raise ValueError(f"q, k, v and cu_seqlens must be on the context's {dev}")
         n = int(total_tokens) * H * HEAD_DIM
         if out is None:
             out = torch.empty((total_tokens, H, HEAD_DIM), dtype=torch.bfloat16, device=q.device)
         else:
             _check_out(out, "out", torch.bfloat16, n, q.device)
-        _check(lib().fp8attn_varlen_fwd_static(
-            self._h, layer, _ptr(q), _ptr(k), _ptr(v), tok_stride, head_stride, _ptr(cu), B,
-            int(max_seqlen), int(total_tokens), H, HEAD_DIM, float(softmax_scale), int(p_rule),
-            _ptr(out), ctypes.c_void_p(_stream(stream, q.device))), "fp8attn_varlen_fwd_static")
+        with torch.cuda.device(dev):
+            _check(lib().fp8attn_varlen_fwd_static(
+                self._h, layer, _ptr(q), _ptr(k), _ptr(v), tok_stride, head_stride, _ptr(cu), B,
+                int(max_seqlen), int(total_tokens), H, HEAD_DIM, float(softmax_scale),
+                int(p_rule), _ptr(out), ctypes.c_void_p(_stream(stream, q.device))),
+                "fp8attn_varlen_fwd_static")
         return out
 
     def quantize_qkv_grouped(self, layer: int, mode: int, q: torch.Tensor, k: torch.Tensor,
